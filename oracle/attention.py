@@ -1,0 +1,279 @@
+"""Plain, slow, fp64 CPU oracle for exact scaled dot-product attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import
+this module.  It shares no code with the CUDA path and imports nothing from
+the ``exact_tiled_attention_31_b200`` package.
+
+What it computes and where the pages define it
+----------------------------------------------
+The method on the pages is *exact* attention: apart from floating-point
+summation order, the tiled kernel returns the plain result
+``O = softmax(Q K^T * scale [+ causal mask]) V`` ("Flash Attention 的算法设计原理"
+(algomooc), "FlashAttention 的定位"; "From Self-Attention to FlashAttention"
+(wmrh.cn), §二 says the online result is numerically equivalent, not an
+approximation).  So the oracle is that definition written out:
+
+* scores ``s_ij = scale * q_i . k_j`` materialised in full
+  ("ops-transformer里的FlashAttention" (mhpn.cn), "FlashAttention的核心思路",
+  step 1 of the conventional flow);
+* the three-pass stable softmax - max, then sum of exponentials, then divide
+  ("From Self-Attention to FlashAttention", §二, first paragraph);
+* ``O = P V`` (same conventional flow, step 3);
+* the per-row log-sum-exp ``LSE_i = m_i + ln l_i`` (natural log of the sum of
+  exponentials of the scaled scores) - the "statistics" the forward keeps so
+  that the backward can rebuild the local blocks ("Flash Attention 的算法设计原理",
+  "核心机制", third item).
+
+The causal mask lets query ``i`` see keys ``j <= i`` (diagonal included,
+top-left aligned; "ops-transformer里的FlashAttention", "实战踩坑 坑二").  In a
+packed variable-length batch each sequence only sees itself, and causality is
+counted from the sequence's own start.
+
+The pages give no backward formulas (only that it recomputes local blocks
+from saved statistics), so the gradients are the textbook ones for
+``L = sum(dO * O)``::
+
+    dV_j  = sum_i P_ij dO_i
+    dP_ij = dO_i . v_j
+    D_i   = sum_j P_ij dP_ij            (= dO_i . O_i)
+    dS_ij = P_ij (dP_ij - D_i)
+    dQ_i  = scale * sum_j dS_ij k_j
+    dK_j  = scale * sum_i dS_ij q_i
+
+Readings where the pages are silent: a row with no visible key (cannot occur
+with equal query/key lengths) returns ``O = 0`` and ``LSE = -inf``.  Large
+inputs are processed a block of query rows at a time; every row still goes
+through its own full three passes, so only memory use changes.
+
+``attention_forward_online`` restates the one-pass running-max / running-sum
+update of "From Self-Attention to FlashAttention", §二 (unnormalised output
+rescaled by ``exp(m_prev - m_new)``, divided once at the end).  It exists
+only so the tests can check that the one-pass form equals the three-pass
+one; the printed update in "ops-transformer里的FlashAttention", "在线softmax",
+divides by the running sum inside the loop and is not used.
+
+All inputs are converted to float64 exactly (bf16/fp16 values are exactly
+representable) before any arithmetic.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "to_f64",
+    "attention_scores",
+    "attention_probs",
+    "attention_forward",
+    "attention_forward_rows",
+    "attention_backward",
+    "attention_forward_online",
+    "varlen_forward",
+    "varlen_backward",
+    "flop_count",
+]
+
+_ROW_BLOCK = 1024
+
+
+def to_f64(x) -> np.ndarray:
+    """Exact conversion of a torch tensor / array of bf16, fp16 or fp32 to float64."""
+    if hasattr(x, "detach"):  # torch tensor, without importing torch here
+        x = x.detach().cpu()
+        if str(x.dtype) in ("torch.bfloat16", "torch.float16"):
+            x = x.float()  # exact widening; numpy has no bfloat16
+        x = x.numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def _visible(nq: int, nk: int, causal: bool, q_rows: np.ndarray | None = None) -> np.ndarray:
+    """Boolean [nq, nk] mask of the keys each query row may attend to."""
+    rows = np.arange(nq) if q_rows is None else np.asarray(q_rows)
+    cols = np.arange(nk)
+    if causal:
+        return cols[None, :] <= rows[:, None]
+    return np.ones((rows.shape[0], nk), dtype=bool)
+
+
+def attention_scores(q: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
+    """s = scale * q k^T for one head: q [Sq, D], k [Sk, D] -> [Sq, Sk]."""
+    return scale * (q @ k.T)
+
+
+def _three_pass(s: np.ndarray, vis: np.ndarray):
+    """Stable softmax of each row over its visible keys, in three passes.
+
+    Returns (P, m, l) with P [rows, keys], m the row maximum and l the sum of
+    exp(s - m) over the visible keys.
+    """
+    masked = np.where(vis, s, -np.inf)
+    m = masked.max(axis=1)                                  # pass 1: maximum
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    e = np.where(vis, np.exp(masked - m_safe[:, None]), 0.0)
+    l = e.sum(axis=1)                                        # pass 2: sum of exp
+    with np.errstate(invalid="ignore", divide="ignore"):
+        p = np.where(l[:, None] > 0, e / l[:, None], 0.0)     # pass 3: divide
+    return p, m, l
+
+
+def attention_probs(q, k, scale: float, causal: bool) -> np.ndarray:
+    """Full probability matrix P for one head (small inputs only)."""
+    q, k = to_f64(q), to_f64(k)
+    s = attention_scores(q, k, scale)
+    p, _, _ = _three_pass(s, _visible(q.shape[0], k.shape[0], causal))
+    return p
+
+
+def _head_forward(q, k, v, scale, causal, rows=None):
+    nq = q.shape[0] if rows is None else len(rows)
+    row_ids = np.arange(q.shape[0]) if rows is None else np.asarray(rows)
+    o = np.zeros((nq, v.shape[1]))
+    lse = np.empty(nq)
+    for b0 in range(0, nq, _ROW_BLOCK):
+        r = row_ids[b0:b0 + _ROW_BLOCK]
+        s = attention_scores(q[r], k, scale)
+        p, m, l = _three_pass(s, _visible(q.shape[0], k.shape[0], causal, r))
+        o[b0:b0 + len(r)] = p @ v
+        with np.errstate(divide="ignore"):
+            lse[b0:b0 + len(r)] = np.where(l > 0, m + np.log(l), -np.inf)
+    return o, lse
+
+
+def attention_forward(q, k, v, scale: float, causal: bool, heads=None):
+    """O and LSE for [B, H, S, D] inputs (or [S, D] for a single head).
+
+    ``heads`` optionally restricts the work to a list of (b, h) pairs; the
+    result then has shape [len(heads), S, D] / [len(heads), S].
+    """
+    q, k, v = to_f64(q), to_f64(k), to_f64(v)
+    if q.ndim == 2:
+        return _head_forward(q, k, v, scale, causal)
+    B, H, S, D = q.shape
+    pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else list(heads)
+    o = np.zeros((len(pairs), S, v.shape[-1]))
+    lse = np.zeros((len(pairs), S))
+    for n, (b, h) in enumerate(pairs):
+        o[n], lse[n] = _head_forward(q[b, h], k[b, h], v[b, h], scale, causal)
+    if heads is None:
+        return o.reshape(B, H, S, -1), lse.reshape(B, H, S)
+    return o, lse
+
+
+def attention_forward_rows(q, k, v, scale: float, causal: bool, b: int, h: int, rows):
+    """O and LSE of selected query rows of head (b, h) - for full-size spot checks."""
+    q, k, v = to_f64(q[b, h]), to_f64(k[b, h]), to_f64(v[b, h])
+    return _head_forward(q, k, v, scale, causal, rows=np.asarray(rows))
+
+
+def _head_backward(q, k, v, do, scale, causal):
+    s = attention_scores(q, k, scale)
+    p, _, _ = _three_pass(s, _visible(q.shape[0], k.shape[0], causal))
+    o = p @ v
+    dv = p.T @ do
+    dp = do @ v.T
+    d_row = (p * dp).sum(axis=1)
+    ds = p * (dp - d_row[:, None])
+    dq = scale * (ds @ k)
+    dk = scale * (ds.T @ q)
+    return dq, dk, dv, o
+
+
+def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None):
+    """dQ, dK, dV of L = sum(dO * O) for [B, H, S, D] (or [S, D]) inputs."""
+    q, k, v, do = to_f64(q), to_f64(k), to_f64(v), to_f64(do)
+    if q.ndim == 2:
+        return _head_backward(q, k, v, do, scale, causal)[:3]
+    B, H, S, D = q.shape
+    pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else list(heads)
+    dq = np.zeros((len(pairs), S, D))
+    dk = np.zeros((len(pairs), S, D))
+    dv = np.zeros((len(pairs), S, v.shape[-1]))
+    for n, (b, h) in enumerate(pairs):
+        dq[n], dk[n], dv[n], _ = _head_backward(q[b, h], k[b, h], v[b, h], do[b, h], scale, causal)
+    if heads is None:
+        return dq.reshape(q.shape), dk.reshape(k.shape), dv.reshape(v.shape)
+    return dq, dk, dv
+
+
+def attention_forward_online(q, k, v, scale: float, causal: bool, block: int = 128):
+    """One-pass online-softmax attention for one head, [S, D] inputs.
+
+    Key/value blocks of ``block`` rows are visited once; for each, every query
+    row updates its running max, rescales its running sum and unnormalised
+    output by exp(m_prev - m_new), and adds the block's contribution; the
+    output is divided by the running sum at the end.
+    """
+    q, k, v = to_f64(q), to_f64(k), to_f64(v)
+    nq, nk = q.shape[0], k.shape[0]
+    o = np.zeros((nq, v.shape[1]))
+    m = np.full(nq, -np.inf)
+    l = np.zeros(nq)
+    for j0 in range(0, nk, block):
+        kj, vj = k[j0:j0 + block], v[j0:j0 + block]
+        s = attention_scores(q, kj, scale)
+        if causal:
+            cols = np.arange(j0, j0 + kj.shape[0])
+            s = np.where(cols[None, :] <= np.arange(nq)[:, None], s, -np.inf)
+        m_new = np.maximum(m, s.max(axis=1))
+        m_ref = np.where(np.isfinite(m_new), m_new, 0.0)
+        corr = np.exp(np.where(np.isfinite(m), m - m_ref, -np.inf))
+        p = np.exp(s - m_ref[:, None])
+        l = corr * l + p.sum(axis=1)
+        o = corr[:, None] * o + p @ vj
+        m = m_new
+    with np.errstate(invalid="ignore", divide="ignore"):
+        out = np.where(l[:, None] > 0, o / l[:, None], 0.0)
+        lse = np.where(l > 0, m + np.log(l), -np.inf)
+    return out, lse
+
+
+def _seq_bounds(cu_seqlens):
+    cu = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    return list(zip(cu[:-1], cu[1:]))
+
+
+def varlen_forward(q, k, v, cu_seqlens, scale: float, causal: bool, heads=None, seqs=None):
+    """Packed [H, T, D] forward: each sequence attends only within itself.
+
+    Returns O [H', T, D] and LSE [H', T] for the heads in ``heads`` (all by
+    default); rows of sequences not in ``seqs`` are left at zero.
+    """
+    q, k, v = to_f64(q), to_f64(k), to_f64(v)
+    H, T, D = q.shape
+    heads = list(range(H)) if heads is None else list(heads)
+    bounds = _seq_bounds(cu_seqlens)
+    seqs = range(len(bounds)) if seqs is None else seqs
+    o = np.zeros((len(heads), T, v.shape[-1]))
+    lse = np.zeros((len(heads), T))
+    for n, h in enumerate(heads):
+        for si in seqs:
+            a, b = bounds[si]
+            o[n, a:b], lse[n, a:b] = _head_forward(q[h, a:b], k[h, a:b], v[h, a:b], scale, causal)
+    return o, lse
+
+
+def varlen_backward(q, k, v, do, cu_seqlens, scale: float, causal: bool, heads=None):
+    """Packed [H, T, D] gradients, one sequence at a time."""
+    q, k, v, do = to_f64(q), to_f64(k), to_f64(v), to_f64(do)
+    H, T, D = q.shape
+    heads = list(range(H)) if heads is None else list(heads)
+    dq = np.zeros((len(heads), T, D))
+    dk = np.zeros((len(heads), T, D))
+    dv = np.zeros((len(heads), T, v.shape[-1]))
+    for n, h in enumerate(heads):
+        for a, b in _seq_bounds(cu_seqlens):
+            dq[n, a:b], dk[n, a:b], dv[n, a:b], _ = _head_backward(
+                q[h, a:b], k[h, a:b], v[h, a:b], do[h, a:b], scale, causal)
+    return dq, dk, dv
+
+
+def flop_count(lengths, heads: int, d: int, causal: bool) -> tuple[float, float]:
+    """(forward, backward) FLOPs by the usual convention.
+
+    Forward counts the two matrix products, 4 * S^2 * D per head, halved
+    under a causal mask; backward counts five products, 2.5x the forward.
+    """
+    f = sum(4.0 * L * L * d for L in lengths) * heads
+    if causal:
+        f *= 0.5
+    return f, 2.5 * f
