@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""Benchmark of exact tiled attention on B200: forward + backward TFLOP/s.
+
+Workload (default): causal bf16 attention, B=1 H=32 S=4096 D=128, scale
+1/sqrt(128), seeded N(0,1) synthetic Q, K, V, dO.  One step is the whole hot
+path: fa_fwd, then the three backward launches (fa_bwd_preprocess,
+fa_bwd_main, fa_bwd_finish).  FLOPs follow the usual convention: forward
+4*B*H*S^2*D halved under the causal mask, backward 2.5x that.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched with torchrun (one rank per GPU).  The heads are
+independent, so every rank runs its own copy of the workload (weak scaling,
+no data-path collective); the NCCL group only carries the barrier and the
+max-over-ranks timing.  ``--impl reference`` times the fp64 CPU oracle on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attn fwd & fwd+bwd TFLOP/s, bf16 causal S=4096 D=128; % of B200 dense peak"
+DATASHEET_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+WORKLOADS = {
+    "b1_h32_s4096_d128_causal": dict(B=1, H=32, S=4096, D=128, causal=True),
+    "b4_h16_s8192_d128_causal": dict(B=4, H=16, S=8192, D=128, causal=True),
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="b1_h32_s4096_d128_causal")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+def flops(w):
+    f = 4.0 * w["B"] * w["H"] * w["S"] ** 2 * w["D"] * (0.5 if w["causal"] else 1.0)
+    return f, 2.5 * f
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads") or 0) for i in threadpool_info())
+        if n:
+            return int(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if gpu_id:
+            cmd += ["-i", gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        self.t0 = self.t1 = None
+
+    def stop(self):
+        if not self.proc:
+            return []
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                stamp, _, frac = parts[0].partition(".")
+                ts = time.mktime(time.strptime(stamp, "%Y/%m/%d %H:%M:%S")) + (float("0." + frac) if frac else 0.0)
+                rows.append(dict(ts=ts, sm=float(parts[1]), sm_max=float(parts[2]),
+                                 power=float(parts[3]) if parts[3] not in ("[N/A]", "N/A") else None,
+                                 reasons=[n for n, v in zip(self.NAMES, parts[4:8]) if v.lower() == "active"]))
+            except (ValueError, IndexError):
+                continue
+        return rows
+
+    def summary(self, rows):
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        inside = [r for r in rows if self.t0 is not None and self.t0 - 0.15 <= r["ts"] <= self.t1 + 0.15]
+        use = inside or rows
+        reasons = sorted({n for r in use for n in r["reasons"]})
+        return {"sm_mhz": statistics.median(r["sm"] for r in use), "sm_max_mhz": max(r["sm_max"] for r in use),
+                "reasons": reasons, "samples": len(use), "samples_in_timed_region": len(inside),
+                "power_w_max": max((r["power"] or 0.0) for r in use)}
+
+
+# ------------------------------------------------------------------ CPU oracle legs
+
+def oracle_sample(w, target_s: float, max_heads: int = 4):
+    """Time the fp64 oracle fwd+bwd on whole heads of the workload until
+    about ``target_s`` seconds have passed; returns (flops, seconds, heads)."""
+    from exact_tiled_attention_31_b200 import inputs
+    from oracle import attention as oa
+    t = inputs.make_dense(1, 1, w["S"], w["D"], "bf16", seed=42, with_do=True)
+    scale = 1.0 / math.sqrt(w["D"])
+    f_fwd, f_bwd = flops(dict(w, B=1, H=1))
+    done, t_total = 0, 0.0
+    while done < max_heads and (done == 0 or t_total < target_s):
+        t0 = time.perf_counter()
+        oa.attention_forward(t["q"][0, 0], t["k"][0, 0], t["v"][0, 0], scale, w["causal"])
+        oa.attention_backward(t["q"][0, 0], t["k"][0, 0], t["v"][0, 0], t["do"][0, 0], scale, w["causal"])
+        t_total += time.perf_counter() - t0
+        done += 1
+    return done * (f_fwd + f_bwd), t_total, done
+
+
+def run_reference(args, rank, world, w):
+    """--impl reference: the fp64 oracle on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    from exact_tiled_attention_31_b200 import inputs
+    from oracle import attention as oa
+    scale = 1.0 / math.sqrt(w["D"])
+    # each step: fwd+bwd of the causal prefix of length L of head (0, 0), L
+    # chosen so the whole run stays within about two minutes
+    t = inputs.make_dense(1, 1, w["S"], w["D"], "bf16", seed=42, with_do=True)
+    q, k, v, do = (t[x][0, 0] for x in ("q", "k", "v", "do"))
+
+    def step(L):
+        oa.attention_forward(q[:L], k[:L], v[:L], scale, w["causal"])
+        oa.attention_backward(q[:L], k[:L], v[:L], do[:L], scale, w["causal"])
+
+    L = w["S"]
+    t0 = time.perf_counter()
+    step(min(L, 512))
+    probe = time.perf_counter() - t0
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    while L > 128 and probe * (L / 512.0) ** 2 > budget:
+        L //= 2
+    for _ in range(args.warmup):
+        step(L)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step(L)
+    el = time.perf_counter() - t0
+    f_fwd, f_bwd = flops(dict(w, B=1, H=1, S=L))
+    val = (f_fwd + f_bwd) * args.steps / el / 1e12
+    sample = f"fwd+bwd of the causal prefix of length {L} of 1 of {w['B'] * w['H']} heads per step"
+    out = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": args.workload, **w},
+           "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def main():
+    args = parse()
+    w = WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world, w)
+        return
+
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import exact_tiled_attention_31_b200 as fa
+    from exact_tiled_attention_31_b200 import inputs
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    B, H, S, D, causal = w["B"], w["H"], w["S"], w["D"], w["causal"]
+    scale = 1.0 / math.sqrt(D)
+    host = inputs.make_dense(B, H, S, D, "bf16", seed=42, with_do=True)
+    q, k, v, do = (host[x].to(dev) for x in ("q", "k", "v", "do"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, S), device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa.fa_bwd_workspace_size(B, H, S, D)
+    ws = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
+    flush = torch.empty(256 * 1024 * 1024, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    dt = fa.api.FA_BF16
+
+    def chk(st, what):
+        if st != 0:
+            raise fa.FAError(st, what)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        chk(fa.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, S, D, scale,
+                      causal, dt, sh), "fa_fwd")
+        if ev:
+            ev[1].record(stream)
+        chk(fa.fa_bwd_preprocess(o.data_ptr(), do.data_ptr(), lse.data_ptr(), B, H, S, D, dt, ws.data_ptr(),
+                                 ws_bytes, sh), "fa_bwd_preprocess")
+        if ev:
+            ev[2].record(stream)
+        chk(fa.fa_bwd_main(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                           B, H, S, D, scale, causal, dt, 0, ws.data_ptr(), ws_bytes, sh), "fa_bwd_main")
+        if ev:
+            ev[3].record(stream)
+        chk(fa.fa_bwd_finish(dq.data_ptr(), B, H, S, D, scale, dt, ws.data_ptr(), ws_bytes, sh), "fa_bwd_finish")
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    fa.check_device_error()
+    torch.cuda.synchronize()
+
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    sampler.t0 = time.time()
+    launches0 = fa.fa_launch_count()
+    for i in range(args.steps):
+        flush.zero_()  # write 256 MiB (> 126 MB L2) between timed steps; not inside any event pair
+        step(evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    sampler.t1 = time.time()
+    launches = fa.fa_launch_count() - launches0
+    clock_rows = sampler.stop()
+    fa.check_device_error()
+
+    t_fwd = [e[0].elapsed_time(e[1]) for e in evs]
+    t_pre = [e[1].elapsed_time(e[2]) for e in evs]
+    t_main = [e[2].elapsed_time(e[3]) for e in evs]
+    t_fin = [e[3].elapsed_time(e[4]) for e in evs]
+    t_step = [e[0].elapsed_time(e[4]) for e in evs]
+    ms = {"step": statistics.mean(t_step), "fwd": statistics.mean(t_fwd), "bwd_pre": statistics.mean(t_pre),
+          "bwd_main": statistics.mean(t_main), "bwd_finish": statistics.mean(t_fin)}
+    if world > 1:
+        tt = torch.tensor([ms[x] for x in ("step", "fwd", "bwd_pre", "bwd_main", "bwd_finish")], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = dict(zip(("step", "fwd", "bwd_pre", "bwd_main", "bwd_finish"), tt.tolist()))
+    f_fwd, f_bwd = flops(w)
+    t_bwd = ms["bwd_pre"] + ms["bwd_main"] + ms["bwd_finish"]
+    value = world * (f_fwd + f_bwd) / (ms["step"] * 1e-3) / 1e12
+    fwd_tf = f_fwd / (ms["fwd"] * 1e-3) / 1e12
+    bwd_tf = f_bwd / (t_bwd * 1e-3) / 1e12
+    fb_tf = (f_fwd + f_bwd) / ((ms["fwd"] + t_bwd) * 1e-3) / 1e12
+
+    # ---- end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (host[x].pin_memory() for x in ("q", "k", "v", "do"))
+        ho = torch.empty_like(hq).pin_memory()
+        hl = torch.empty((B, H, S), dtype=torch.float32).pin_memory()
+        hdq, hdk, hdv = (torch.empty_like(hq).pin_memory() for _ in range(3))
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
+        d2h = sum(x.numel() * x.element_size() for x in (ho, hl, hdq, hdk, hdv))
+        e_steps = max(3, min(args.steps, 20))
+
+        def e2e_step():
+            dq_ = torch.empty_like(q)
+            for hsrc, dst in ((hq, q), (hk, k), (hv, v), (hdo, do)):
+                dst.copy_(hsrc, non_blocking=True)
+            o_, l_ = fa.forward(q, k, v, causal, scale, out=o, lse=lse)
+            g = fa.backward(q, k, v, o_, do, l_, causal, scale, workspace=ws)
+            for src, hdst in ((o_, ho), (l_, hl), (g[0], hdq), (g[1], hdk), (g[2], hdv)):
+                hdst.copy_(src, non_blocking=True)
+            del dq_
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / e_steps
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = tt.item()
+        e2e = {"value": world * (f_fwd + f_bwd) / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "api": "exact_tiled_attention_31_b200.forward/backward (ctypes over libfa.so)"}
+
+    # ---- roofline of the dominant kernel
+    pk, pk_kind = peaks()
+    dominant = "bwd_main" if ms["bwd_main"] >= ms["fwd"] else "fwd"
+    alg = f_bwd if dominant == "bwd_main" else f_fwd
+    achieved = alg / (ms[dominant] * 1e-3) / 1e12
+    roofline = {"kernel": "fa::bwd_main_kernel<128,bf16,causal>" if dominant == "bwd_main"
+                else "fa::fwd_kernel<128,bf16,causal,dense>",
+                "bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                "peak_source": f"{pk_kind} bf16 dense burst (MEASURED_PEAKS.json bf16_tflops)"
+                if pk_kind == "measured" else "fallback 1590 TFLOP/s (no MEASURED_PEAKS.json)",
+                "algorithmic_flops_per_launch": alg, "ms_per_launch": ms[dominant]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        fl, sec, nh = oracle_sample(w, target_s=10.0)
+        cpu = {"value": fl / sec / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"fp64 fwd+bwd of {nh} of {B * H} heads (full S={S}), {sec:.1f} s"}
+
+    clocks = sampler.summary(clock_rows)
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms["step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, **w, "scale": scale, "seed": 42,
+                       "l2": "flushed between timed steps (256 MiB write)",
+                       "parallelism": f"replicas x{world} (independent heads, no data-path collective)"},
+            "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf, "fwd_bwd_tflops": fb_tf,
+            "fwd_pct_of_2250": 100 * fwd_tf / DATASHEET_TFLOPS, "bwd_pct_of_2250": 100 * bwd_tf / DATASHEET_TFLOPS,
+            "fwd_bwd_pct_of_2250": 100 * fb_tf / DATASHEET_TFLOPS,
+            "fwd_frac_of_measured": fwd_tf / pk["bf16_tflops"], "bwd_frac_of_measured": bwd_tf / pk["bf16_tflops"],
+            "kernel_ms": ms, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": clocks,
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

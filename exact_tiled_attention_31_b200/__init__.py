@@ -1,0 +1,12 @@
+"""Exact tiled attention for NVIDIA B200 (sm_100a).
+
+The CUDA kernels live in ``libfa.so`` (built from ``csrc/`` by
+``exact_tiled_attention_31_b200.build``); ``api`` is a thin ctypes binding
+over its C ABI (``include/fa.h``).  ``inputs`` draws the seeded synthetic
+tensors used by the tests and the benchmark.
+"""
+from .api import (  # noqa: F401
+    EXPORTS, FAError, backward, check_device_error, fa_bwd, fa_bwd_finish, fa_bwd_main, fa_bwd_preprocess,
+    fa_bwd_workspace_size, fa_check_device_error,
+    fa_fwd, fa_fwd_varlen, fa_launch_count, fa_status_string, forward, forward_varlen, load_library,
+)

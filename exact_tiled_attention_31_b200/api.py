@@ -1,0 +1,210 @@
+"""ctypes binding of libfa.so (include/fa.h).
+
+Two layers:
+
+* ``fa_fwd``, ``fa_fwd_varlen``, ``fa_bwd_workspace_size``, ``fa_bwd``,
+  ``fa_status_string``, ``fa_check_device_error``, ``fa_launch_count``: the C
+  entry points under the same names, taking raw device pointers (ints) and
+  sizes, returning the ``fa_status`` code.
+* ``forward``, ``forward_varlen``, ``backward``: tensor conveniences that
+  check shapes/dtypes, allocate outputs and workspace with torch (device
+  memory and the current stream are all torch provides) and raise
+  ``FAError`` on a non-zero status.
+
+Every step of the attention itself runs in the library's CUDA kernels; there
+is no fallback.  If ``libfa.so`` is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+FA_BF16, FA_FP16 = 0, 1
+
+EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
+           "fa_bwd_finish", "fa_status_string", "fa_check_device_error", "fa_launch_count")
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {fa_status_string(status)} ({status})")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libfa.so once; raise loudly if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m exact_tiled_attention_31_b200.build` "
+            "(there is no non-CUDA implementation to fall back to)")
+    lib = ctypes.CDLL(path)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+    lib.fa_fwd.restype = i
+    lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+    lib.fa_fwd_varlen.restype = i
+    lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_bwd_workspace_size.restype = sz
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp, sz, vp]
+    lib.fa_bwd.restype = i
+    lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, i, i, i, i, i, vp, sz, vp]
+    lib.fa_bwd_preprocess.restype = i
+    lib.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp, sz, vp]
+    lib.fa_bwd_main.restype = i
+    lib.fa_bwd_finish.argtypes = [vp, i, i, i, i, f, i, vp, sz, vp]
+    lib.fa_bwd_finish.restype = i
+    lib.fa_status_string.argtypes = [i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_check_device_error.argtypes = [vp]
+    lib.fa_check_device_error.restype = i
+    lib.fa_launch_count.argtypes = []
+    lib.fa_launch_count.restype = ctypes.c_uint64
+    _lib = lib
+    return lib
+
+
+# ---------------------------------------------------------------- raw entry points
+
+def fa_fwd(q, k, v, o, lse, B, H, S, D, scale, causal, dt, stream) -> int:
+    return load_library().fa_fwd(q, k, v, o, lse, B, H, S, D, scale, int(causal), dt, stream)
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, nseq, max_seqlen, total, H, D, scale, causal, dt, stream) -> int:
+    return load_library().fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, nseq, max_seqlen, total, H, D, scale,
+                                        int(causal), dt, stream)
+
+
+def fa_bwd_workspace_size(B, H, S, D) -> int:
+    return load_library().fa_bwd_workspace_size(B, H, S, D)
+
+
+def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, causal, dt, deterministic, workspace,
+           workspace_bytes, stream) -> int:
+    return load_library().fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, int(causal), dt,
+                                 int(deterministic), workspace, workspace_bytes, stream)
+
+
+def fa_bwd_preprocess(o, dO, lse, B, H, S, D, dt, workspace, workspace_bytes, stream) -> int:
+    return load_library().fa_bwd_preprocess(o, dO, lse, B, H, S, D, dt, workspace, workspace_bytes, stream)
+
+
+def fa_bwd_main(q, k, v, dO, dk, dv, B, H, S, D, scale, causal, dt, deterministic, workspace, workspace_bytes,
+                stream) -> int:
+    return load_library().fa_bwd_main(q, k, v, dO, dk, dv, B, H, S, D, scale, int(causal), dt, int(deterministic),
+                                      workspace, workspace_bytes, stream)
+
+
+def fa_bwd_finish(dq, B, H, S, D, scale, dt, workspace, workspace_bytes, stream) -> int:
+    return load_library().fa_bwd_finish(dq, B, H, S, D, scale, dt, workspace, workspace_bytes, stream)
+
+
+def fa_status_string(status: int) -> str:
+    return load_library().fa_status_string(status).decode()
+
+
+def fa_check_device_error(stream) -> int:
+    return load_library().fa_check_device_error(stream)
+
+
+def fa_launch_count() -> int:
+    return load_library().fa_launch_count()
+
+
+# ---------------------------------------------------------------- tensor conveniences
+
+def _dt(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float16:
+        return FA_FP16
+    raise TypeError(f"expected bf16 or fp16 tensors, got {t.dtype}")
+
+
+def _check(ts, shape):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"shape {tuple(t.shape)} != {tuple(shape)}")
+        if t.dtype != ts[0].dtype:
+            raise TypeError("all tensors must share one dtype")
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def forward(q, k, v, causal: bool, scale: float | None = None, out=None, lse=None, stream=None):
+    """O, LSE of [B, H, S, D] inputs; LSE is fp32 [B, H, S]."""
+    import torch
+    B, H, S, D = q.shape
+    _check((q, k, v), q.shape)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, S), device=q.device, dtype=torch.float32) if lse is None else lse
+    st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, S, D, scale,
+                causal, _dt(q), _stream(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd")
+    return o, lse
+
+
+def forward_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool, scale: float | None = None,
+                   stream=None):
+    """Packed [H, T, D] forward; ``cu_seqlens`` is a device int32 tensor."""
+    import torch
+    H, T, D = q.shape
+    _check((q, k, v), q.shape)
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
+        raise TypeError("cu_seqlens must be a CUDA int32 tensor")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    o = torch.empty_like(q)
+    lse = torch.empty((H, T), device=q.device, dtype=torch.float32)
+    st = fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                       cu_seqlens.data_ptr(), cu_seqlens.numel() - 1, int(max_seqlen), T, H, D, scale, causal,
+                       _dt(q), _stream(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_varlen")
+    return o, lse
+
+
+def backward(q, k, v, o, do, lse, causal: bool, scale: float | None = None, deterministic: bool = False,
+             workspace=None, stream=None):
+    """dQ, dK, dV of [B, H, S, D] inputs given the forward's O and LSE."""
+    import torch
+    B, H, S, D = q.shape
+    _check((q, k, v, o, do), q.shape)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nbytes = fa_bwd_workspace_size(B, H, S, D)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(max(nbytes, 1), device=q.device, dtype=torch.uint8)
+    st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, S, D, scale, causal, _dt(q), deterministic,
+                workspace.data_ptr(), workspace.numel(), _stream(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def check_device_error(stream=None):
+    """Synchronise and raise FAError if a kernel recorded a timeout."""
+    st = fa_check_device_error(_stream(stream))
+    if st != FA_OK:
+        raise FAError(st, "device")

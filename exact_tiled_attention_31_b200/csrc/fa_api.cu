@@ -1,0 +1,342 @@
+// fa_api.cu - host side of the C ABI declared in include/fa.h: argument
+// checks, TMA tensor-map encoding, launch configuration and the device error
+// word.  All device work happens in the kernels of fa_fwd.cuh / fa_bwd.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <initializer_list>
+
+#include "../../include/fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// [heads, rows, D] 16-bit tensor, boxes of 128 rows x 64 columns, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int D, long long rows, long long heads, bool bf16) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
+
+// Opt every kernel instance into its dynamic shared memory once per device
+// (one flag word per instance: the template argument is the kernel itself).
+template <auto Kernel>
+cudaError_t set_smem(uint32_t bytes) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load() & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done.fetch_or(bit);
+  return e;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+fa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+// ---------------------------------------------------------------- forward
+template <int D, bool BF16, bool CAUSAL, bool VARLEN>
+fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
+                     cudaStream_t st) {
+  using C = fa::FwdCfg<D>;
+  auto kern = fa::fwd_kernel<D, BF16, CAUSAL, VARLEN>;
+  cudaError_t e = set_smem<fa::fwd_kernel<D, BF16, CAUSAL, VARLEN>>(C::SMEM);
+  if (e != cudaSuccess) return FA_ERR_CUDA;
+  const long long grid = (long long)p.n_pairs * p.nseq * p.heads;
+  if (grid <= 0) return FA_OK;
+  if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  kern<<<(unsigned)grid, C::THREADS, C::SMEM, st>>>(mq, mk, mv, p);
+  g_launches.fetch_add(1);
+  return from_cuda(cudaGetLastError());
+}
+
+template <int D, bool BF16>
+fa_status dispatch_fwd(bool causal, bool varlen, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const fa::FwdParams& p, cudaStream_t st) {
+  if (varlen)
+    return causal ? launch_fwd<D, BF16, true, true>(mq, mk, mv, p, st)
+                  : launch_fwd<D, BF16, false, true>(mq, mk, mv, p, st);
+  return causal ? launch_fwd<D, BF16, true, false>(mq, mk, mv, p, st)
+                : launch_fwd<D, BF16, false, false>(mq, mk, mv, p, st);
+}
+
+fa_status run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu, int heads,
+                  int seqlen, long long rows, int nseq, int D, float scale, bool causal, bool bf16, bool varlen,
+                  cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, D, rows, heads, bf16) || !make_map(&mk, k, D, rows, heads, bf16) ||
+      !make_map(&mv, v, D, rows, heads, bf16))
+    return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.cu_seqlens = cu;
+  p.heads = heads;
+  p.seqlen = seqlen;
+  p.rows = (int)rows;
+  p.nseq = nseq;
+  p.n_pairs = (seqlen + 255) / 256;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (D == 64)
+    return bf16 ? dispatch_fwd<64, true>(causal, varlen, mq, mk, mv, p, st)
+                : dispatch_fwd<64, false>(causal, varlen, mq, mk, mv, p, st);
+  return bf16 ? dispatch_fwd<128, true>(causal, varlen, mq, mk, mv, p, st)
+              : dispatch_fwd<128, false>(causal, varlen, mq, mk, mv, p, st);
+}
+
+// ---------------------------------------------------------------- backward
+struct WsLayout {
+  size_t dq_acc, lse2, delta, sem, total;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WsLayout ws_layout(long long heads, long long S, int D) {
+  const long long n_q = (S + 127) / 128, S_pad = n_q * 128;
+  WsLayout w;
+  w.dq_acc = 0;
+  w.lse2 = up256((size_t)heads * S * D * 4);
+  w.delta = w.lse2 + up256((size_t)heads * S_pad * 4);
+  w.sem = w.delta + up256((size_t)heads * S_pad * 4);
+  w.total = w.sem + up256((size_t)heads * n_q * 4);
+  return w;
+}
+
+fa::BwdParams bwd_params(int heads, int S, int D, float scale, int deterministic, uint8_t* ws, void* dk, void* dv) {
+  const WsLayout w = ws_layout(heads, S, D);
+  fa::BwdParams p;
+  p.dk = dk;
+  p.dv = dv;
+  p.dq_acc = reinterpret_cast<float*>(ws + w.dq_acc);
+  p.lse2 = p.lse2_w = reinterpret_cast<float*>(ws + w.lse2);
+  p.delta = p.delta_w = reinterpret_cast<float*>(ws + w.delta);
+  p.sem = reinterpret_cast<uint32_t*>(ws + w.sem);
+  p.heads = heads;
+  p.S = S;
+  p.n_q = (S + 127) / 128;
+  p.S_pad = p.n_q * 128;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.deterministic = deterministic;
+  return p;
+}
+
+template <int D, bool BF16>
+fa_status launch_bwd_pre(const void* o, const void* dO, const float* lse, const fa::BwdParams& p, cudaStream_t st) {
+  fa::bwd_pre_kernel<D, BF16><<<sm_count() * 8, 256, 0, st>>>(static_cast<const uint16_t*>(o),
+                                                                static_cast<const uint16_t*>(dO), lse, p);
+  g_launches.fetch_add(1);
+  return from_cuda(cudaGetLastError());
+}
+
+template <int D, bool BF16>
+fa_status launch_bwd_main(const void* q, const void* k, const void* v, const void* dO, const fa::BwdParams& p,
+                          bool causal, cudaStream_t st) {
+  using C = fa::BwdCfg<D>;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, q, D, p.S, p.heads, BF16) || !make_map(&mk, k, D, p.S, p.heads, BF16) ||
+      !make_map(&mv, v, D, p.S, p.heads, BF16) || !make_map(&mdo, dO, D, p.S, p.heads, BF16))
+    return FA_ERR_CUDA;
+  const long long grid = (long long)p.n_q * p.heads;
+  if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  cudaError_t e = causal ? set_smem<fa::bwd_main_kernel<D, BF16, true>>(C::SMEM)
+                         : set_smem<fa::bwd_main_kernel<D, BF16, false>>(C::SMEM);
+  if (e != cudaSuccess) return FA_ERR_CUDA;
+  if (causal)
+    fa::bwd_main_kernel<D, BF16, true><<<(unsigned)grid, 384, C::SMEM, st>>>(mq, mk, mv, mdo, p);
+  else
+    fa::bwd_main_kernel<D, BF16, false><<<(unsigned)grid, 384, C::SMEM, st>>>(mq, mk, mv, mdo, p);
+  g_launches.fetch_add(1);
+  return from_cuda(cudaGetLastError());
+}
+
+template <bool BF16>
+fa_status launch_bwd_post(void* dq, const fa::BwdParams& p, int D, cudaStream_t st) {
+  const long long n8 = (long long)p.heads * p.S * D / 8;
+  fa::bwd_post_kernel<BF16><<<sm_count() * 8, 256, 0, st>>>(p.dq_acc, static_cast<uint16_t*>(dq), n8, p.scale);
+  g_launches.fetch_add(1);
+  return from_cuda(cudaGetLastError());
+}
+
+// shared checks of the backward entry points: sizes, dtype, workspace
+fa_status bwd_common_checks(int B, int H, int S, int D, fa_dtype dt, const void* workspace, size_t workspace_bytes) {
+  if (B < 0 || H < 0 || S < 0) return FA_ERR_INVALID_ARG;
+  if (dt != FA_BF16 && dt != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * H > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || S == 0) return FA_OK;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_INVALID_ARG;
+  size_t need = ws_layout((long long)B * H, S, D).total;
+  if (workspace_bytes < need) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+bool ptrs_ok(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (!p || !aligned16(p)) return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int D,
+                 float scale, int causal, fa_dtype dt, void* stream) {
+  if (B < 0 || H < 0 || S < 0) return FA_ERR_INVALID_ARG;
+  if (dt != FA_BF16 && dt != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || S == 0) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  const long long heads = (long long)B * H;
+  if (heads > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  return run_fwd(q, k, v, o, lse, nullptr, (int)heads, S, S, 1, D, scale, causal != 0, dt == FA_BF16, false,
+                 static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens,
+                        int nseq, int max_seqlen, int total, int H, int D, float scale, int causal, fa_dtype dt,
+                        void* stream) {
+  if (nseq < 0 || max_seqlen < 0 || total < 0 || H < 0) return FA_ERR_INVALID_ARG;
+  if (dt != FA_BF16 && dt != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (nseq == 0 || H == 0 || total == 0 || max_seqlen == 0) return FA_OK;
+  if (max_seqlen > total) return FA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse || !cu_seqlens) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return FA_ERR_INVALID_ARG;
+  return run_fwd(q, k, v, o, lse, cu_seqlens, H, max_seqlen, total, nseq, D, scale, causal != 0, dt == FA_BF16, true,
+                 static_cast<cudaStream_t>(stream));
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int S, int D) {
+  if (B <= 0 || H <= 0 || S <= 0 || (D != 64 && D != 128)) return 0;
+  return ws_layout((long long)B * H, S, D).total;
+}
+
+fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int S, int D,
+                            fa_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
+  fa_status c = bwd_common_checks(B, H, S, D, dt, workspace, workspace_bytes);
+  if (c != FA_OK || B == 0 || H == 0 || S == 0) return c;
+  if (!ptrs_ok({o, dO, lse})) return FA_ERR_INVALID_ARG;
+  const fa::BwdParams p = bwd_params(B * H, S, D, 1.f, 0, static_cast<uint8_t*>(workspace), nullptr, nullptr);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 64) return dt == FA_BF16 ? launch_bwd_pre<64, true>(o, dO, lse, p, st) : launch_bwd_pre<64, false>(o, dO, lse, p, st);
+  return dt == FA_BF16 ? launch_bwd_pre<128, true>(o, dO, lse, p, st) : launch_bwd_pre<128, false>(o, dO, lse, p, st);
+}
+
+fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B, int H,
+                      int S, int D, float scale, int causal, fa_dtype dt, int deterministic, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  fa_status c = bwd_common_checks(B, H, S, D, dt, workspace, workspace_bytes);
+  if (c != FA_OK) return c;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || S == 0) return FA_OK;
+  if (!ptrs_ok({q, k, v, dO, dk, dv})) return FA_ERR_INVALID_ARG;
+  const fa::BwdParams p =
+      bwd_params(B * H, S, D, scale, deterministic != 0, static_cast<uint8_t*>(workspace), dk, dv);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool cz = causal != 0;
+  if (D == 64)
+    return dt == FA_BF16 ? launch_bwd_main<64, true>(q, k, v, dO, p, cz, st) : launch_bwd_main<64, false>(q, k, v, dO, p, cz, st);
+  return dt == FA_BF16 ? launch_bwd_main<128, true>(q, k, v, dO, p, cz, st) : launch_bwd_main<128, false>(q, k, v, dO, p, cz, st);
+}
+
+fa_status fa_bwd_finish(void* dq, int B, int H, int S, int D, float scale, fa_dtype dt, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  fa_status c = bwd_common_checks(B, H, S, D, dt, workspace, workspace_bytes);
+  if (c != FA_OK) return c;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || S == 0) return FA_OK;
+  if (!ptrs_ok({dq})) return FA_ERR_INVALID_ARG;
+  const fa::BwdParams p = bwd_params(B * H, S, D, scale, 0, static_cast<uint8_t*>(workspace), nullptr, nullptr);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dt == FA_BF16 ? launch_bwd_post<true>(dq, p, D, st) : launch_bwd_post<false>(dq, p, D, st);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int H, int S, int D, float scale, int causal, fa_dtype dt,
+                 int deterministic, void* workspace, size_t workspace_bytes, void* stream) {
+  fa_status c = bwd_common_checks(B, H, S, D, dt, workspace, workspace_bytes);
+  if (c != FA_OK) return c;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || S == 0) return FA_OK;
+  if (!ptrs_ok({q, k, v, o, dO, lse, dq, dk, dv})) return FA_ERR_INVALID_ARG;
+  c = fa_bwd_preprocess(o, dO, lse, B, H, S, D, dt, workspace, workspace_bytes, stream);
+  if (c != FA_OK) return c;
+  c = fa_bwd_main(q, k, v, dO, dk, dv, B, H, S, D, scale, causal, dt, deterministic, workspace, workspace_bytes,
+                  stream);
+  if (c != FA_OK) return c;
+  return fa_bwd_finish(dq, B, H, S, D, scale, dt, workspace, workspace_bytes, stream);
+}
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: null, misaligned or out-of-range argument";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: head dim or size not implemented";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a kernel gave up waiting on an internal barrier";
+  }
+  return "unknown fa_status";
+}
+
+fa_status fa_check_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  uint32_t code = 0;
+  if (cudaMemcpyFromSymbol(&code, fa::g_dev_error, sizeof(code)) != cudaSuccess) return FA_ERR_CUDA;
+  if (code == 0) return FA_OK;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(fa::g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+  return FA_ERR_TIMEOUT;
+}
+
+uint64_t fa_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,158 @@
+/*
+ * fa.h - C ABI of the exact tiled attention library (libfa.so) for NVIDIA B200 (sm_100a).
+ *
+ * The library computes exact scaled dot-product attention
+ *
+ *     O = softmax(Q K^T * scale [+ causal mask]) V
+ *
+ * tile by tile with an online softmax, so the S x S score and probability
+ * matrices never reach device memory ("From Self-Attention to FlashAttention",
+ * §一 flowchart and §二 Online Softmax; "ops-transformer里的FlashAttention",
+ * "FlashAttention的核心思路").  The forward keeps only the per-row log-sum-exp,
+ * and the backward rebuilds each local probability block from it
+ * ("Flash Attention 的算法设计原理", "核心机制", third item).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are dense, row-major, 16-bit (bf16 or fp16 as chosen by `dt`) in
+ *    device memory owned by the caller.  The library never allocates,
+ *    frees or keeps a pointer across calls.
+ *  - Dense layout: [B, H, S, D] contiguous (D innermost).  LSE: fp32 [B, H, S].
+ *  - Packed variable-length layout: [H, T, D] contiguous, T = total tokens;
+ *    sequence s occupies token rows cu_seqlens[s] .. cu_seqlens[s+1]-1.
+ *    LSE: fp32 [H, T].
+ *  - Every base pointer must be 16-byte aligned (the kernels move tiles with
+ *    the Tensor Memory Accelerator).
+ *  - Supported head dims: D = 64 or 128.  S (or each sequence) may be any
+ *    length >= 1; ragged tails are handled inside the kernels.
+ *  - causal != 0 lets query i attend keys j <= i (diagonal included, counted
+ *    from the start of each sequence), as the causal flag of the operator in
+ *    "ops-transformer里的FlashAttention", "ops-transformer里的完整算子" and
+ *    "实战踩坑 坑二".
+ *  - scale is applied to Q K^T (normally 1/sqrt(D)); it must be finite and > 0.
+ *  - All calls are asynchronous on `stream` (a cudaStream_t, 0 = legacy
+ *    default stream).  Argument errors are reported synchronously before
+ *    anything is launched; launch failures return FA_ERR_CUDA.  A kernel that
+ *    waits too long on one of its internal barriers gives up, records
+ *    FA_ERR_TIMEOUT in a per-device error word and exits; read it with
+ *    fa_check_device_error().
+ *  - No entry point falls back to another implementation: unsupported
+ *    arguments return FA_ERR_UNSUPPORTED.
+ */
+#ifndef EXACT_TILED_ATTENTION_FA_H
+#define EXACT_TILED_ATTENTION_FA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, bad scale */
+  FA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. D not in {64,128}) */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  FA_ERR_TIMEOUT = 4      /* a kernel gave up waiting on an internal barrier */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/*
+ * Forward pass.
+ *   q, k, v : [B, H, S, D] inputs (read only).
+ *   o       : [B, H, S, D] output, same dtype.
+ *   lse     : [B, H, S] fp32 output, natural-log log-sum-exp of each row's
+ *             scaled scores (the statistic the backward recomputes P from).
+ * Cites: "From Self-Attention to FlashAttention", §二 (running max / running
+ * sum update, final division); "ops-transformer里的FlashAttention",
+ * "核心计算流程" (Q tile resident, K/V tiles streamed, only O written back).
+ * B, H or S equal to 0 is a no-op returning FA_OK.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int S, int D, float scale, int causal, fa_dtype dt,
+                 void* stream);
+
+/*
+ * Forward pass over a packed batch of variable-length sequences.
+ *   q, k, v, o : [H, total, D];  lse : fp32 [H, total].
+ *   cu_seqlens : DEVICE int32 [nseq + 1], cu_seqlens[0] = 0, non-decreasing,
+ *                cu_seqlens[nseq] = total.
+ *   max_seqlen : an upper bound on every sequence length (sizes the grid).
+ * Each sequence attends only within itself.  Cites: "Flash Attention 的算法设计原理",
+ * "练习口述回答" (variable-length inputs are a branch to cover on their own).
+ * The library does not read cu_seqlens on the host; offsets that break the
+ * stated rules give unspecified (but in-bounds) results.
+ */
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens, int nseq, int max_seqlen, int total,
+                        int H, int D, float scale, int causal, fa_dtype dt, void* stream);
+
+/*
+ * Bytes of device scratch that fa_bwd needs for these sizes: an fp32 dQ
+ * accumulator [B, H, S, D], the fp32 row terms D_i = dO_i . O_i [B, H, S],
+ * and the ordering counters of deterministic mode, each 256-byte aligned.
+ * Returns 0 for unsupported sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int S, int D);
+
+/*
+ * Backward pass.  Inputs q, k, v, o, dO ([B, H, S, D]) and lse ([B, H, S],
+ * from fa_fwd); outputs dq, dk, dv ([B, H, S, D], same dtype).
+ * workspace: caller-owned device buffer of at least
+ * fa_bwd_workspace_size(B, H, S, D) bytes, 256-byte aligned; its contents on
+ * entry do not matter and are overwritten.
+ * deterministic = 0: dQ partial sums from different key tiles are added with
+ *   fp32 atomics, so dq may differ in the last bits from run to run.
+ * deterministic = 1: the key tiles of one query tile add their dQ partials in
+ *   increasing key-tile order, so repeated calls with the same inputs, sizes
+ *   and GPU give bit-identical dq (the `deterministic` option of the
+ *   operator config in "ops-transformer里的FlashAttention", "ops-transformer里的完整算子").
+ * The gradients are those of L = sum(dO * O): dV = P^T dO, dS = P o (dP - D),
+ * dQ = scale dS K, dK = scale dS^T Q, with P rebuilt from lse
+ * ("Flash Attention 的算法设计原理", "核心机制"; the pages print no formulas, these
+ * are the textbook ones).
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv,
+                 int B, int H, int S, int D, float scale, int causal, fa_dtype dt,
+                 int deterministic, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The three launches fa_bwd makes, exposed for callers that want to place
+ * or time them separately (same arguments, same rules, same workspace; they
+ * must run in this order on one stream):
+ *   fa_bwd_preprocess  D_i = dO_i . O_i and LSE * log2(e) into the
+ *                      workspace; clears the dQ accumulator and the
+ *                      deterministic-mode counters.
+ *   fa_bwd_main        the tiled pass over key/value tiles: writes dk, dv
+ *                      and accumulates unscaled dQ (fp32) in the workspace.
+ *   fa_bwd_finish      dq = scale * accumulated dQ, rounded to the dtype.
+ */
+fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int S, int D,
+                            fa_dtype dt, void* workspace, size_t workspace_bytes, void* stream);
+fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                      int B, int H, int S, int D, float scale, int causal, fa_dtype dt, int deterministic,
+                      void* workspace, size_t workspace_bytes, void* stream);
+fa_status fa_bwd_finish(void* dq, int B, int H, int S, int D, float scale, fa_dtype dt,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* A static, human-readable name for a status code. */
+const char* fa_status_string(fa_status s);
+
+/*
+ * Synchronises `stream`, then reads and clears the calling device's error
+ * word.  Returns FA_OK, FA_ERR_TIMEOUT (a kernel gave up waiting) or
+ * FA_ERR_CUDA (the synchronisation itself failed).
+ */
+fa_status fa_check_device_error(void* stream);
+
+/* Number of kernel launches issued by this process through the library so far. */
+uint64_t fa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_TILED_ATTENTION_FA_H */

@@ -1,0 +1,60 @@
+"""Shared helpers for the GPU parity tests: tolerances and comparisons.
+
+Tolerances (written here once, used by every parity test):
+  O    : max |O_gpu - O_ref| <= 1e-2 and mean |O_gpu - O_ref| <= 1e-3
+  LSE  : max |LSE_gpu - LSE_ref| <= 1e-3
+  dQ, dK, dV : max |G_gpu - G_ref| <= 2e-2 * max |G_ref|   (each tensor on its own)
+The references are the fp64 oracle on the identical 16-bit inputs.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+O_MAX, O_MEAN, LSE_MAX, GRAD_REL = 1e-2, 1e-3, 1e-3, 2e-2
+
+
+def f64(t) -> np.ndarray:
+    if isinstance(t, np.ndarray):
+        return t.astype(np.float64)
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def check_o(o_gpu, o_ref, what=""):
+    o_gpu, o_ref = f64(o_gpu), f64(o_ref)
+    assert np.isfinite(o_gpu).all(), f"{what}: non-finite O"
+    err = np.abs(o_gpu - o_ref)
+    emax, emean = err.max(), err.mean()
+    if emax > O_MAX or emean > O_MEAN:
+        idx = np.unravel_index(err.argmax(), err.shape)
+        raise AssertionError(f"{what}: O max-abs {emax:.3e} (limit {O_MAX}) mean-abs {emean:.3e} "
+                             f"(limit {O_MEAN}); worst at {idx}: gpu {o_gpu[idx]:.5f} ref {o_ref[idx]:.5f}")
+    return emax, emean
+
+
+def check_lse(l_gpu, l_ref, what=""):
+    l_gpu, l_ref = f64(l_gpu), f64(l_ref)
+    assert np.isfinite(l_gpu).all(), f"{what}: non-finite LSE"
+    err = np.abs(l_gpu - l_ref)
+    if err.max() > LSE_MAX:
+        idx = np.unravel_index(err.argmax(), err.shape)
+        raise AssertionError(f"{what}: LSE max-abs {err.max():.3e} (limit {LSE_MAX}); worst at {idx}: "
+                             f"gpu {l_gpu[idx]:.6f} ref {l_ref[idx]:.6f}")
+    return err.max()
+
+
+def check_grad(g_gpu, g_ref, name):
+    g_gpu, g_ref = f64(g_gpu), f64(g_ref)
+    assert np.isfinite(g_gpu).all(), f"{name}: non-finite values"
+    scale = np.abs(g_ref).max()
+    err = np.abs(g_gpu - g_ref).max()
+    rel = err / scale if scale > 0 else err
+    if rel > GRAD_REL:
+        idx = np.unravel_index(np.abs(g_gpu - g_ref).argmax(), g_ref.shape)
+        raise AssertionError(f"{name}: max-abs {err:.3e} = {rel:.3e} x max|ref| {scale:.3e} (limit {GRAD_REL}); "
+                             f"worst at {idx}: gpu {g_gpu[idx]:.5f} ref {g_ref[idx]:.5f}")
+    return rel
+
+
+def to_dev(t: dict, dev) -> dict:
+    return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in t.items()}

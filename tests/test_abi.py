@@ -1,0 +1,96 @@
+"""CPU-side checks of the C ABI: the library loads without a GPU, exports
+every function include/fa.h declares, and rejects bad arguments before it
+touches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_tiled_attention_31_b200 as fa
+from exact_tiled_attention_31_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_library()
+    return fa.load_library()
+
+
+def _declared():
+    names = set()
+    for hdr in os.listdir(os.path.join(ROOT, "include")):
+        text = open(os.path.join(ROOT, "include", hdr)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert {"fa_fwd", "fa_fwd_varlen", "fa_bwd", "fa_bwd_workspace_size"} <= names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(fa.EXPORTS) <= names
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        assert fa.fa_status_string(code).startswith("FA_")
+
+
+def test_workspace_size_formula(lib):
+    def up(x):
+        return (x + 255) // 256 * 256
+    for B, H, S, D in [(1, 32, 4096, 128), (2, 3, 17, 64), (4, 16, 8192, 128)]:
+        heads, spad = B * H, (S + 127) // 128 * 128
+        expect = up(heads * S * D * 4) + 2 * up(heads * spad * 4) + up(heads * (spad // 128) * 4)
+        assert fa.fa_bwd_workspace_size(B, H, S, D) == expect
+    assert fa.fa_bwd_workspace_size(1, 1, 16, 96) == 0
+    assert fa.fa_bwd_workspace_size(0, 1, 16, 64) == 0
+
+
+def test_fwd_argument_errors(lib):
+    A = 1 << 20  # a 16-byte aligned fake address, never dereferenced
+    ok = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=1, S=16, D=64, scale=0.125, causal=0, dt=0, stream=None)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return fa.fa_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["S"], a["D"], a["scale"],
+                         a["causal"], a["dt"], a["stream"])
+    assert call(D=96) == fa.api.FA_ERR_UNSUPPORTED
+    assert call(D=256) == fa.api.FA_ERR_UNSUPPORTED
+    assert call(S=-1) == fa.api.FA_ERR_INVALID_ARG
+    assert call(dt=7) == fa.api.FA_ERR_INVALID_ARG
+    assert call(scale=0.0) == fa.api.FA_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == fa.api.FA_ERR_INVALID_ARG
+    assert call(q=0) == fa.api.FA_ERR_INVALID_ARG
+    assert call(o=A + 8) == fa.api.FA_ERR_INVALID_ARG
+    assert call(B=0) == fa.api.FA_OK      # empty problem: nothing to do
+    assert call(S=0, q=0) == fa.api.FA_OK
+
+
+def test_varlen_and_bwd_argument_errors(lib):
+    A = 1 << 20
+    assert fa.fa_fwd_varlen(A, A, A, A, A, A, 2, 300, 100, 1, 64, 0.1, 1, 0, None) == fa.api.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_varlen(A, A, A, A, A, A + 2, 2, 50, 100, 1, 64, 0.1, 1, 0, None) == fa.api.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_varlen(A, A, A, A, A, A, 2, 50, 100, 1, 80, 0.1, 1, 0, None) == fa.api.FA_ERR_UNSUPPORTED
+    assert fa.fa_fwd_varlen(A, A, A, A, A, A, 0, 50, 100, 1, 64, 0.1, 1, 0, None) == fa.api.FA_OK
+    need = fa.fa_bwd_workspace_size(1, 1, 64, 64)
+    args = [A] * 9 + [1, 1, 64, 64, 0.125, 1, 0, 0]
+    assert fa.fa_bwd(*args, A, need - 1, None) == fa.api.FA_ERR_INVALID_ARG      # workspace too small
+    assert fa.fa_bwd(*args, A + 16, need, None) == fa.api.FA_ERR_INVALID_ARG     # workspace not 256-aligned
+    assert fa.fa_bwd(*([A] * 8 + [0]), 1, 1, 64, 64, 0.125, 1, 0, 0, A, need, None) == fa.api.FA_ERR_INVALID_ARG
+    assert fa.fa_bwd(*([A] * 9), 1, 1, 64, 48, 0.125, 1, 0, 0, A, need, None) == fa.api.FA_ERR_UNSUPPORTED
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    saved = fa.api._lib
+    fa.api._lib = None
+    try:
+        with pytest.raises(RuntimeError, match="missing"):
+            fa.api.load_library(str(tmp_path / "nope.so"))
+    finally:
+        fa.api._lib = saved
