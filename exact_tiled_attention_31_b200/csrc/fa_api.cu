@@ -48,6 +48,20 @@ bool make_map(CUtensorMap* m, const void* base, int D, long long rows, long long
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 dQ accumulator [heads, rows, D] for TMA bulk reductions: boxes of
+// 32 rows x 32 columns (128 bytes), 128-byte swizzle.
+bool make_map_f32(CUtensorMap* m, const void* base, int D, long long rows, long long heads) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)rows * D * 4};
+  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
@@ -175,9 +189,10 @@ template <int D, bool BF16>
 fa_status launch_bwd_main(const void* q, const void* k, const void* v, const void* dO, const fa::BwdParams& p,
                           bool causal, cudaStream_t st) {
   using C = fa::BwdCfg<D>;
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   if (!make_map(&mq, q, D, p.S, p.heads, BF16) || !make_map(&mk, k, D, p.S, p.heads, BF16) ||
-      !make_map(&mv, v, D, p.S, p.heads, BF16) || !make_map(&mdo, dO, D, p.S, p.heads, BF16))
+      !make_map(&mv, v, D, p.S, p.heads, BF16) || !make_map(&mdo, dO, D, p.S, p.heads, BF16) ||
+      !make_map_f32(&mdq, p.dq_acc, D, p.S, p.heads))
     return FA_ERR_CUDA;
   const long long grid = (long long)p.n_q * p.heads;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
@@ -185,9 +200,9 @@ fa_status launch_bwd_main(const void* q, const void* k, const void* v, const voi
                          : set_smem<fa::bwd_main_kernel<D, BF16, false>>(C::SMEM);
   if (e != cudaSuccess) return FA_ERR_CUDA;
   if (causal)
-    fa::bwd_main_kernel<D, BF16, true><<<(unsigned)grid, 384, C::SMEM, st>>>(mq, mk, mv, mdo, p);
+    fa::bwd_main_kernel<D, BF16, true><<<(unsigned)grid, 384, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, p);
   else
-    fa::bwd_main_kernel<D, BF16, false><<<(unsigned)grid, 384, C::SMEM, st>>>(mq, mk, mv, mdo, p);
+    fa::bwd_main_kernel<D, BF16, false><<<(unsigned)grid, 384, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, p);
   g_launches.fetch_add(1);
   return from_cuda(cudaGetLastError());
 }

@@ -16,23 +16,33 @@
 //             into a 128-row-padded copy, zero the fp32 dQ accumulator and
 //             the ordering counters.
 //   bwd_main  one CTA per 128-row key/value tile j of one head (384 threads):
-//               warp 0     TMA producer: K_j, V_j once; then dO_i and Q_i
-//                          (plus the padded LSE/D rows of tile i) through a
-//                          ring of three shared-memory slots.
-//               warp 1     tcgen05 issuer and TMEM owner.  Per query tile i:
-//                            dP^T = V_j dO_i^T        -> TMEM [128,256)
-//                            S^T  = K_j Q_i^T         -> TMEM [0,128)
-//                            dV  += P^T dO_i   (P^T from TMEM)  -> [256,256+D)
-//                            dK  += dS^T Q_i   (dS^T from TMEM) -> [256+D,256+2D)
-//                            dQ_i = dS K_j     (dS from smem)   -> TMEM [0,D)
-//               warps 4-7  one thread per key row: P^T = exp2(S^T*scale*log2e
-//                          - LSE*log2e), dS^T = P^T (dP^T - D) in one pass over
-//                          32-column chunks; P^T and dS^T go back to TMEM as
-//                          16-bit pairs, dS also to shared memory (the A operand
-//                          of the dQ product); at the end dV and scale*dK.
-//               warps 8-11 one thread per query row: drain dQ_i from TMEM and
-//                          add it to the fp32 accumulator (fp32 atomics, or in
-//                          key-tile order under deterministic mode).
+//               warp 0     TMA producer: K_j, V_j once; then Q_i (+ the padded
+//                          LSE/D rows of tile i) into a 2-slot ring and dO_i
+//                          into its own slot.
+//               warp 1     tcgen05 issuer and TMEM owner.  TMEM columns:
+//                          A = [0,128): S^T, then P^T (16-bit) in [0,64)
+//                          B = [128,256): dP^T, then dS^T in [0,64), then dQ_i
+//                          dV [256,256+D), dK [256+D,256+2D).
+//                          Issue order for query tile i (one step):
+//                            dV  += P^T dO_i          (A = P^T in TMEM)
+//                            S^T(i+1) = K_j Q_{i+1}^T  -> A
+//                            dK  += dS^T Q_i          (A = dS^T in TMEM)
+//                            dQ_i = dS K_j            (A = dS in smem) -> B
+//                            dP^T(i+1) = V_j dO_{i+1}^T -> B (after dQ_i left TMEM)
+//                          so the exponentials of tile i+1 run while the
+//                          tensor core does dK_i, dQ_i and dP^T(i+1).
+//               warps 4-7  one thread per key row.  P phase: P^T =
+//                          exp2(S^T*scale*log2e - LSE*log2e), kept as 16-bit
+//                          pairs in registers and written to TMEM A.  dS
+//                          phase: dS^T = P^T (dP^T - D) to TMEM B and, as the
+//                          MN-major A operand of dQ = dS K, to shared memory.
+//                          At the end: dV and scale*dK rows to global memory.
+//               warps 8-11 one thread per query row: move dQ_i from TMEM to a
+//                          per-warp 128-byte-swizzled staging buffer and add it
+//                          to the fp32 accumulator with TMA bulk reductions
+//                          (cp.reduce.async.bulk.tensor .add); under
+//                          deterministic mode instead, key tiles add into query
+//                          tile i one at a time in increasing j.
 //   bwd_post  dQ = scale * accumulator, rounded to the input dtype.
 // Causal: key tile j only meets query tiles i >= j; only the diagonal tile
 // is masked element-wise.
@@ -59,25 +69,27 @@ struct BwdParams {
 template <int D>
 struct BwdCfg {
   static constexpr int CH = D / 64;
-  static constexpr uint32_t CHUNK = 128u * 128u;
-  static constexpr uint32_t TILE = CH * CHUNK;
-  static constexpr int NSLOT = 3;                        // ring for dO_i / Q_i
+  static constexpr uint32_t CHUNK = 128u * 128u;                // 128 rows x 128 bytes
+  static constexpr uint32_t TILE = CH * CHUNK;                   // one 128 x D 16-bit tile
   static constexpr uint32_t K_OFF = 0;
   static constexpr uint32_t V_OFF = TILE;
-  static constexpr uint32_t RING_OFF = 2 * TILE;
-  static constexpr uint32_t DS_OFF = RING_OFF + NSLOT * TILE;   // 128 x 128 16-bit, 2 chunks
-  static constexpr uint32_t STAT_OFF = DS_OFF + 2 * CHUNK;      // NSLOT x (128 lse2 + 128 delta) fp32
-  static constexpr uint32_t BAR_OFF = STAT_OFF + NSLOT * 1024;
-  // kv_full ring_full[3] ring_empty[3] s_full dp_full pds_full dq_full dq_empty dkv_full drain dq_done
-  static constexpr int NBAR = 1 + 2 * NSLOT + 8;
+  static constexpr uint32_t Q_OFF = 2 * TILE;                    // 2 slots
+  static constexpr uint32_t DO_OFF = 4 * TILE;                   // 1 slot
+  static constexpr uint32_t DS_OFF = 5 * TILE;                   // 128 x 128 16-bit, 2 chunks
+  static constexpr uint32_t STG_OFF = DS_OFF + 2 * CHUNK;        // 4 warps x (32 rows x 128 B) fp32 staging
+  static constexpr uint32_t STAT_OFF = STG_OFF + 4 * 4096;       // 2 slots x (128 lse2 + 128 delta) fp32
+  static constexpr uint32_t BAR_OFF = STAT_OFF + 2 * 1024;
+  // kv_full q_full[2] q_empty[2] do_full do_empty s_full dp_full p_full ds_full
+  // dq_full dq_empty dkv_full drain dq_done
+  static constexpr int NBAR = 17;
   static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
-  static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D, TM_DQ = 0;
+  static constexpr uint32_t TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
 };
 
 enum : uint32_t {
-  BWD_SITE_PROD = 0x200, BWD_SITE_KV = 0x201, BWD_SITE_RING = 0x202, BWD_SITE_PDS = 0x203,
-  BWD_SITE_DQE = 0x204, BWD_SITE_S = 0x205, BWD_SITE_DQF = 0x206, BWD_SITE_DKV = 0x207,
-  BWD_SITE_SEM = 0x208, BWD_SITE_DRAIN = 0x209, BWD_SITE_STAT = 0x20a
+  BWD_SITE_PROD = 0x200, BWD_SITE_KV = 0x201, BWD_SITE_Q = 0x202, BWD_SITE_DO = 0x203, BWD_SITE_P = 0x204,
+  BWD_SITE_DS = 0x205, BWD_SITE_DQE = 0x206, BWD_SITE_S = 0x207, BWD_SITE_DP = 0x208, BWD_SITE_DQF = 0x209,
+  BWD_SITE_DKV = 0x20a, BWD_SITE_SEM = 0x20b, BWD_SITE_DRAIN = 0x20c, BWD_SITE_STAT = 0x20d
 };
 
 // ---------------------------------------------------------------------------
@@ -153,6 +165,19 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// fp32 tile in shared memory added element-wise into global memory by the
+// TMA unit (bulk-group completion).
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, const void* src, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(src))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -169,9 +194,9 @@ template <int D, bool BF16, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<D>;
-  const int j = blockIdx.x / p.heads;       // key/value tile (ascending: longest causal work first)
+  const int j = blockIdx.x / p.heads;  // key/value tile (ascending: longest causal work first)
   const int head = blockIdx.x - j * p.heads;
   const int i_begin = CAUSAL ? j : 0;
   const int n_steps = p.n_q - i_begin;
@@ -181,16 +206,19 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* kv_full = bars;
-  uint64_t* ring_full = bars + 1;
-  uint64_t* ring_empty = ring_full + C::NSLOT;
-  uint64_t* s_full = ring_empty + C::NSLOT;
-  uint64_t* dp_full = s_full + 1;
-  uint64_t* pds_full = dp_full + 1;
-  uint64_t* dq_full = pds_full + 1;
-  uint64_t* dq_empty = dq_full + 1;
-  uint64_t* dkv_full = dq_empty + 1;
-  uint64_t* drain = dkv_full + 1;
-  uint64_t* dq_done = drain + 1;
+  uint64_t* q_full = bars + 1;    // [2]
+  uint64_t* q_empty = bars + 3;   // [2]
+  uint64_t* do_full = bars + 5;
+  uint64_t* do_empty = bars + 6;
+  uint64_t* s_full = bars + 7;
+  uint64_t* dp_full = bars + 8;
+  uint64_t* p_full = bars + 9;
+  uint64_t* ds_full = bars + 10;
+  uint64_t* dq_full = bars + 11;
+  uint64_t* dq_empty = bars + 12;
+  uint64_t* dkv_full = bars + 13;
+  uint64_t* drain = bars + 14;
+  uint64_t* dq_done = bars + 15;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   float* stats = reinterpret_cast<float*>(smem + C::STAT_OFF);
 
@@ -199,13 +227,16 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int i = 0; i < C::NSLOT; ++i) {
-      mbar_init(&ring_full[i], 1);
-      mbar_init(&ring_empty[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
     }
+    mbar_init(do_full, 1);
+    mbar_init(do_empty, 1);
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(pds_full, 128);
+    mbar_init(p_full, 128);
+    mbar_init(ds_full, 128);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
     mbar_init(dkv_full, 1);
@@ -234,31 +265,32 @@ __global__ void __launch_bounds__(384, 1)
         tma_load_3d(smem + C::K_OFF + c * C::CHUNK, &tm_k, kv_full, c * 64, kv_row0, head);
         tma_load_3d(smem + C::V_OFF + c * C::CHUNK, &tm_v, kv_full, c * 64, kv_row0, head);
       }
-      uint32_t fill = 0;
       bool ok = true;
+      int q_issued = 0, do_issued = 0;
       for (int st = 0; st < n_steps && ok; ++st) {
         const int i = i_begin + st;
-        for (int which = 0; which < 2; ++which) {  // 0: dO_i, 1: Q_i (+ its LSE/D rows)
-          const uint32_t slot = fill % C::NSLOT, round = fill / C::NSLOT;
-          if (round > 0 && !mbar_wait(&ring_empty[slot], (round - 1) & 1, BWD_SITE_PROD)) {
-            ok = false;
-            break;
-          }
-          mbar_expect_tx(&ring_full[slot], C::TILE + (which ? 1024u : 0u));
-          for (int c = 0; c < C::CH; ++c)
-            tma_load_3d(smem + C::RING_OFF + slot * C::TILE + c * C::CHUNK, which ? &tm_q : &tm_do, &ring_full[slot],
-                        c * 64, 128 * i, head);
-          if (which) {
-            const size_t srow = (size_t)head * p.S_pad + 128 * i;
-            bulk_load(stats + slot * 256, p.lse2 + srow, 512, &ring_full[slot]);
-            bulk_load(stats + slot * 256 + 128, p.delta + srow, 512, &ring_full[slot]);
-          }
-          ++fill;
-        }
+        // Q_i and its LSE / D rows into Q slot st % 2
+        const int qs = st & 1;
+        if (st >= 2 && !(ok = mbar_wait(&q_empty[qs], ((st >> 1) - 1) & 1, BWD_SITE_PROD))) break;
+        mbar_expect_tx(&q_full[qs], C::TILE + 1024u);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(smem + C::Q_OFF + qs * C::TILE + c * C::CHUNK, &tm_q, &q_full[qs], c * 64, 128 * i, head);
+        const size_t srow = (size_t)head * p.S_pad + 128 * i;
+        bulk_load(stats + qs * 256, p.lse2 + srow, 512, &q_full[qs]);
+        bulk_load(stats + qs * 256 + 128, p.delta + srow, 512, &q_full[qs]);
+        ++q_issued;
+        // dO_i into the dO slot
+        if (st >= 1 && !(ok = mbar_wait(do_empty, (st - 1) & 1, BWD_SITE_PROD))) break;
+        mbar_expect_tx(do_full, C::TILE);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(smem + C::DO_OFF + c * C::CHUNK, &tm_do, do_full, c * 64, 128 * i, head);
+        ++do_issued;
       }
-      for (uint32_t f = (fill > (uint32_t)C::NSLOT ? fill - C::NSLOT : 0); f < fill; ++f)
-        mbar_wait(&ring_full[f % C::NSLOT], (f / C::NSLOT) & 1, BWD_SITE_PROD);
+      // no tile copy may still be landing in shared memory at exit
       mbar_wait(kv_full, 0, BWD_SITE_PROD);
+      for (int u = (q_issued > 2 ? q_issued - 2 : 0); u < q_issued; ++u)
+        mbar_wait(&q_full[u & 1], (u >> 1) & 1, BWD_SITE_PROD);
+      if (do_issued > 0) mbar_wait(do_full, (do_issued - 1) & 1, BWD_SITE_PROD);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -268,66 +300,63 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t ID_TS = make_idesc(128, D, BF16, false, true);     // dV, dK
       constexpr uint32_t ID_DQ = make_idesc(128, D, BF16, true, true);      // dQ
       const uint32_t sk = smem_addr(smem + C::K_OFF), sv = smem_addr(smem + C::V_OFF);
-      const uint32_t sring = smem_addr(smem + C::RING_OFF), sds = smem_addr(smem + C::DS_OFF);
-      bool ok = mbar_wait(kv_full, 0, BWD_SITE_KV);
-      uint32_t use = 0;
-      for (int st = 0; st < n_steps && ok; ++st) {
-        const uint32_t so = use % C::NSLOT;
-        if (!(ok = mbar_wait(&ring_full[so], (use / C::NSLOT) & 1, BWD_SITE_RING))) break;
-        ++use;
-        const uint32_t sqs = use % C::NSLOT;
-        // dP^T = V dO^T  (M = keys, N = queries, K = D; both K-major)
-        {
-          const uint32_t da = sring + so * C::TILE;
+      const uint32_t sq = smem_addr(smem + C::Q_OFF), sdo = smem_addr(smem + C::DO_OFF);
+      const uint32_t sds = smem_addr(smem + C::DS_OFF);
+      // X^T = A_kv B_q^T with both operands K-major (X = S or dP)
+      auto kk_product = [&](uint32_t d_col, uint32_t a, uint32_t b) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-            mma_ss(tmem + C::TM_DP, make_sdesc(sv + off, 16, 1024), make_sdesc(da + off, 16, 1024), ID_KK, kk > 0);
-          }
-          mma_commit(dp_full);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          mma_ss(tmem + d_col, make_sdesc(a + off, 16, 1024), make_sdesc(b + off, 16, 1024), ID_KK, kk > 0);
         }
-        if (!(ok = mbar_wait(&ring_full[sqs], (use / C::NSLOT) & 1, BWD_SITE_RING))) break;
-        ++use;
-        // the previous dQ_i has left TMEM [0, D)
-        if (st > 0 && !(ok = mbar_wait(dq_empty, (st - 1) & 1, BWD_SITE_DQE))) break;
+      };
+      bool ok = mbar_wait(kv_full, 0, BWD_SITE_KV) && mbar_wait(&q_full[0], 0, BWD_SITE_Q) &&
+                mbar_wait(do_full, 0, BWD_SITE_DO);
+      if (ok) {
+        kk_product(C::TM_A, sk, sq);  // S^T(0)
+        mma_commit(s_full);
+        kk_product(C::TM_B, sv, sdo);  // dP^T(0)
+        mma_commit(dp_full);
+      }
+      for (int st = 0; st < n_steps && ok; ++st) {
+        const int qs = st & 1;
+        // dV += P^T dO_i
+        if (!(ok = mbar_wait(p_full, st & 1, BWD_SITE_P))) break;
         tc_fence_after();
-        // S^T = K Q^T
-        {
-          const uint32_t qa = sring + sqs * C::TILE;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-            mma_ss(tmem + C::TM_S, make_sdesc(sk + off, 16, 1024), make_sdesc(qa + off, 16, 1024), ID_KK, kk > 0);
-          }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + C::TM_DV, tmem + C::TM_A + kk * 8, make_sdesc(sdo + kk * 2048, C::CHUNK, 1024), ID_TS,
+                 (st > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(do_empty);
+        // S^T(i+1) into A (P^T(i) has been read by the products above)
+        const bool more = st + 1 < n_steps;
+        if (more) {
+          if (!(ok = mbar_wait(&q_full[qs ^ 1], ((st + 1) >> 1) & 1, BWD_SITE_Q))) break;
+          kk_product(C::TM_A, sk, sq + (qs ^ 1) * C::TILE);
           mma_commit(s_full);
         }
-        if (!(ok = mbar_wait(pds_full, st & 1, BWD_SITE_PDS))) break;
+        // dK += dS^T Q_i
+        if (!(ok = mbar_wait(ds_full, st & 1, BWD_SITE_DS))) break;
         tc_fence_after();
-        // dV += P^T dO  (A = P^T in TMEM [0,64), B = dO MN-major)
-        {
-          const uint32_t da = sring + so * C::TILE;
+        const uint32_t qa = sq + qs * C::TILE;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8, make_sdesc(da + kk * 2048, C::CHUNK, 1024), ID_TS,
-                   (st > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&ring_empty[so]);
-        }
-        // dK += dS^T Q  (A = dS^T in TMEM [128,192), B = Q MN-major)
-        {
-          const uint32_t qa = sring + sqs * C::TILE;
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + C::TM_DK, tmem + C::TM_B + kk * 8, make_sdesc(qa + kk * 2048, C::CHUNK, 1024), ID_TS,
+                 (st > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&q_empty[qs]);
+        // dQ_i = dS K_j into B  (A = dS MN-major in smem, B = K MN-major)
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + C::TM_DK, tmem + C::TM_DP + kk * 8, make_sdesc(qa + kk * 2048, C::CHUNK, 1024), ID_TS,
-                   (st > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&ring_empty[sqs]);
-        }
-        // dQ_i = dS K  (M = queries: A = dS MN-major in smem; B = K MN-major)
-        {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + C::TM_DQ, make_sdesc(sds + kk * 2048, C::CHUNK, 1024),
-                   make_sdesc(sk + kk * 2048, C::CHUNK, 1024), ID_DQ, kk > 0);
-          mma_commit(dq_full);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + C::TM_B, make_sdesc(sds + kk * 2048, C::CHUNK, 1024),
+                 make_sdesc(sk + kk * 2048, C::CHUNK, 1024), ID_DQ, kk > 0);
+        mma_commit(dq_full);
+        // dP^T(i+1) into B once dQ_i has been drained
+        if (more) {
+          if (!(ok = mbar_wait(dq_empty, st & 1, BWD_SITE_DQE))) break;
+          if (!(ok = mbar_wait(do_full, (st + 1) & 1, BWD_SITE_DO))) break;
+          tc_fence_after();
+          kk_product(C::TM_B, sv, sdo);
+          mma_commit(dp_full);
         }
       }
       mma_commit(dkv_full);
@@ -339,6 +368,7 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------------------ P / dS (one thread per key row)
     const int r = threadIdx.x - 128;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tA = tmem + lane_off + C::TM_A, tB = tmem + lane_off + C::TM_B;
     const int kv = kv_row0 + r;
     const bool kv_valid = kv < p.S;
     const float sl2 = p.scale_log2;
@@ -346,55 +376,71 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int st = 0; st < n_steps; ++st) {
       const int i = i_begin + st;
-      const uint32_t use_q = 2 * st + 1;
-      ok = mbar_wait(s_full, st & 1, BWD_SITE_S);
-      ok = ok && mbar_wait(dp_full, st & 1, BWD_SITE_S);
-      ok = ok && mbar_wait(&ring_full[use_q % C::NSLOT], (use_q / C::NSLOT) & 1, BWD_SITE_STAT);
+      const int qs = st & 1;
+      ok = mbar_wait(s_full, st & 1, BWD_SITE_S) && mbar_wait(&q_full[qs], (st >> 1) & 1, BWD_SITE_STAT);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const float* lse2 = stats + (use_q % C::NSLOT) * 256;
+      const float* lse2 = stats + qs * 256;
       const float* dlt = lse2 + 128;
       // visible queries of this key row in tile i: q >= kv under the causal mask
       const int qlo = (CAUSAL && i == j) ? r : 0;
-#pragma unroll 1
+      // ---- P phase
+      uint32_t pk[64];
+#pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32(tmem + lane_off + C::TM_S + 32 * ch, sv);
-        tmem_ld32(tmem + lane_off + C::TM_DP + 32 * ch, dv);
+        uint32_t sv[32];
+        tmem_ld32(tA + 32 * ch, sv);
         tmem_ld_wait(sv);
-        tmem_ld_wait(dv);
-        uint32_t pp[16], dd[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float pr[2], dsr[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = 32 * ch + 2 * e + u;
-            float pe = ex2(fmaf(__uint_as_float(sv[2 * e + u]), sl2, -lse2[c]));
-            if (c < qlo || !kv_valid) pe = 0.f;
-            pr[u] = pe;
-            dsr[u] = pe * (__uint_as_float(dv[2 * e + u]) - dlt[c]);
-          }
-          pp[e] = pack2<BF16>(pr[0], pr[1]);
-          dd[e] = pack2<BF16>(dsr[0], dsr[1]);
+          const int c = 32 * ch + 2 * e;
+          float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -lse2[c]));
+          float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -lse2[c + 1]));
+          if (c < qlo || !kv_valid) p0 = 0.f;
+          if (c + 1 < qlo || !kv_valid) p1 = 0.f;
+          pk[16 * ch + e] = pack2<BF16>(p0, p1);
         }
-        tmem_st16(tmem + lane_off + C::TM_S + 16 * ch, pp);
-        tmem_st16(tmem + lane_off + C::TM_DP + 16 * ch, dd);
+      }
+      {
+        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
+        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
+        tmem_st32(tA, lo);
+        tmem_st32(tA + 32, hi);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+      // ---- dS phase
+      ok = __all_sync(0xffffffffu, mbar_wait(dp_full, st & 1, BWD_SITE_DP));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t dv[32];
+        tmem_ld32(tB + 32 * ch, dv);
+        tmem_ld_wait(dv);
+        uint32_t dd[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c = 32 * ch + 2 * e;
+          const float2 pp = unpack2<BF16>(pk[16 * ch + e]);
+          dd[e] = pack2<BF16>(pp.x * (__uint_as_float(dv[2 * e]) - dlt[c]),
+                              pp.y * (__uint_as_float(dv[2 * e + 1]) - dlt[c + 1]));
+        }
+        tmem_st16(tB + 16 * ch, dd);
         // dS row r (key) holds 32 query columns of chunk ch: MN-major A operand
         // of dQ = dS K, i.e. [key][query] with queries contiguous, 128-B swizzled.
-        const uint32_t colbyte = (ch & 1) * 64;               // 32 queries = 64 B inside the 128-B row
-        const uint32_t base = (ch >> 1) * C::CHUNK + r * 128;  // 64-query chunk, key row
+        const uint32_t base = (ch >> 1) * C::CHUNK + r * 128 + (ch & 1) * 64;
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4) {
-          const uint32_t off = swz128(base + colbyte + v4 * 16);
-          *reinterpret_cast<uint4*>(ds_smem + off) = make_uint4(dd[4 * v4], dd[4 * v4 + 1], dd[4 * v4 + 2], dd[4 * v4 + 3]);
-        }
+        for (int v4 = 0; v4 < 4; ++v4)
+          *reinterpret_cast<uint4*>(ds_smem + swz128(base + v4 * 16)) =
+              make_uint4(dd[4 * v4], dd[4 * v4 + 1], dd[4 * v4 + 2], dd[4 * v4 + 3]);
       }
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(pds_full);
+      mbar_arrive(ds_full);
     }
     // ---- epilogue: dV and scale * dK rows of this key tile
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dkv_full, 0, BWD_SITE_DKV));
@@ -411,37 +457,56 @@ __global__ void __launch_bounds__(384, 1)
           uint32_t ov[32];
           tmem_ld32(tmem + lane_off + col + 32 * cc, ov);
           tmem_ld_wait(ov);
-          uint32_t pk[16];
+          uint32_t pkk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            pk[e] = pack2<BF16>(__uint_as_float(ov[2 * e]) * mul, __uint_as_float(ov[2 * e + 1]) * mul);
+            pkk[e] = pack2<BF16>(__uint_as_float(ov[2 * e]) * mul, __uint_as_float(ov[2 * e + 1]) * mul);
           if (kv_valid) {
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              dst[cc * 4 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+              dst[cc * 4 + e] = make_uint4(pkk[4 * e], pkk[4 * e + 1], pkk[4 * e + 2], pkk[4 * e + 3]);
           }
         }
       }
     }
   } else if (warp >= 8) {
-    // ------------------------------------------------------------ dQ drain (one thread per query row)
-    const int c = threadIdx.x - 256;
+    // ------------------------------------------------------------ dQ (one thread per query row)
+    const int c = threadIdx.x - 256;                 // query row within the tile = TMEM lane
+    const int wq = warp - 8;                         // this warp's 32 rows: 32*wq ..
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    uint8_t* stg = smem + C::STG_OFF + wq * 4096;    // 32 rows x 128 B, 128-B swizzled
+    if (!p.deterministic && lane == 0) tma_prefetch_desc(&tm_dq);
     for (int st = 0; st < n_steps; ++st) {
       const int i = i_begin + st;
       if (!__all_sync(0xffffffffu, mbar_wait(dq_full, st & 1, BWD_SITE_DQF))) break;
       tc_fence_after();
       uint32_t a[D / 32][32];
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tmem + lane_off + C::TM_DQ + 32 * cc, a[cc]);
+      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tmem + lane_off + C::TM_B + 32 * cc, a[cc]);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) tmem_ld_wait(a[cc]);
       tc_fence_before();
       mbar_arrive(dq_empty);
       const int q = 128 * i + c;
-      uint32_t* sem = p.sem + (size_t)head * p.n_q + i;
-      if (p.deterministic) {
+      if (!p.deterministic) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          if (lane == 0) bulk_wait_read0();  // the previous reduction has read the buffer
+          __syncwarp();
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            *reinterpret_cast<uint4*>(stg + swz128(lane * 128 + v4 * 16)) =
+                make_uint4(a[cc][4 * v4], a[cc][4 * v4 + 1], a[cc][4 * v4 + 2], a[cc][4 * v4 + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_3d(&tm_dq, stg, 32 * cc, 128 * i + 32 * wq, head);
+            bulk_commit();
+          }
+        }
+      } else {
         // key tiles add into query tile i in increasing j: wait for our turn
+        uint32_t* sem = p.sem + (size_t)head * p.n_q + i;
         bool ok = true;
         if (ld_acquire_gpu(sem) != (uint32_t)j) {
           const uint64_t t0 = global_ns();
@@ -477,17 +542,10 @@ __global__ void __launch_bounds__(384, 1)
             st_release_gpu(sem, (uint32_t)j + 1);
           }
         }
-      } else if (q < p.S) {
-        float4* dst = reinterpret_cast<float4*>(p.dq_acc + ((size_t)head * p.S + q) * D);
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc)
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            atomicAdd(&dst[cc * 8 + e], make_float4(__uint_as_float(a[cc][4 * e]), __uint_as_float(a[cc][4 * e + 1]),
-                                                     __uint_as_float(a[cc][4 * e + 2]),
-                                                     __uint_as_float(a[cc][4 * e + 3])));
       }
     }
+    if (lane == 0) bulk_wait0();  // every reduction issued by this warp has completed
+    __syncwarp();
   }
 
   tc_fence_before();

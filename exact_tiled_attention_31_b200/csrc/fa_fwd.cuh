@@ -22,8 +22,11 @@
 //               per row (TMEM lane); scores are taken to the log2 domain
 //               (scale * log2 e) and exponentiated with ex2; P is written
 //               back into the first 64 columns of the S_t it came from, as
-//               packed 16-bit pairs; O_t is rescaled in TMEM when the row
-//               max grows; at the end O_t / l and LSE go to global memory.
+//               packed 16-bit pairs; O_t and the running sums are rescaled
+//               when the row max grows (the TMEM loads of O_t are issued
+//               ahead of the exponentials that hide them); the sum that
+//               normalises O adds the P values as rounded for the P V
+//               product; at the end O_t / l and LSE go to global memory.
 //   The two query tiles ping-pong: while one softmax group works, the
 //   tensor core runs the other tile's products.
 // TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
@@ -61,6 +64,11 @@ struct FwdCfg {
   static constexpr uint32_t TM_S = 0, TM_O = 256;
   static constexpr int THREADS = 384;
 };
+
+// Row-max growth (log2 units) tolerated before O and l are rescaled.  Zero
+// keeps the exact running max, so the dominant P of every row is exactly 1
+// and only the smaller weights carry 16-bit rounding into P V.
+constexpr float kRescaleLog2 = 0.f;
 
 // wait-site ids reported through the error word
 enum : uint32_t {
@@ -141,6 +149,11 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t sq = smem_addr(smem + C::Q_OFF);
   const uint32_t skv = smem_addr(smem + C::KV_OFF);
 
+  // register split: 128 x 56 (warps 0-3) + 256 x 208 (softmax) = 60416 <= 384 x 168.
+  // Each warpgroup changes its budget inside its own branch so the compiler
+  // allocates every role with the budget it runs under.
+  if (warp < 4) {
+  regs_dec<56>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -262,7 +275,9 @@ __global__ void __launch_bounds__(384, 1)
       mbar_wait(drain, 0, FWD_SITE_DRAIN);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_inc<208>();
     // ------------------------------------------------------------ softmax
     const int t = (warp - 4) >> 2;
     const int n_t = t == 0 ? n0 : n1;
@@ -272,7 +287,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tO = tmem + lane_off + C::TM_O + D * t;
     const int row = q_start + 128 * t + r;  // row inside the sequence
     const float sl2 = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f, lr = 0.f;
     bool ok = true;
     for (int j = 0; j < n_t; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, FWD_SITE_S));
@@ -307,59 +322,76 @@ __global__ void __launch_bounds__(384, 1)
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(fmaxf(x0[c], x1[c]), fmaxf(x2[c], x3[c])));
-      const float m_new = fmaxf(m, mx * sl2);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2(m - m_use);
-      const float neg = -m_use;
-      float sum0 = 0.f, sum1 = 0.f;
+      // Rescale O and the running sums only when the row max actually grew
+      // (by more than kRescaleLog2): every P is then <= 2^kRescaleLog2, and
+      // with kRescaleLog2 = 0 the largest P of the row is exactly 1.
+      const float m_max = fmaxf(m, mx * sl2);
+      const bool rescale = m_max > m + kRescaleLog2;  // false while the row has no visible key
+      const float m_new = rescale ? m_max : m;
+      const float alpha = rescale ? ex2(m - m_new) : 1.f;  // ex2(-inf) = 0 on the first tile
+      const float neg = (m_new == -INFINITY) ? 0.f : -m_new;
+      const uint64_t scale2 = f2(sl2, sl2), neg2 = f2(neg, neg);
+      // fsum: fp32 sum of P (for LSE); rsum: sum of P as rounded to 16 bits
+      // (the weights the P V product uses, for normalising O).
+      uint64_t fsum = f2(0.f, 0.f), rsum = f2(0.f, 0.f);
+      auto exp_pack = [&](float x, float y) -> uint32_t {
+        float a, b;
+        f2split(ffma2(f2(x, y), scale2, neg2), a, b);
+        a = ex2(a);
+        b = ex2(b);
+        fsum = fadd2(fsum, f2(a, b));
+        const uint32_t pk = pack2<BF16>(a, b);
+        rsum = fadd2(rsum, widen2<BF16>(pk));
+        return pk;
+      };
+      // O_t (written by the previous P V product, complete once S_t arrived)
+      // is rescaled 32 columns at a time, each load issued one exponential
+      // chunk ahead so its latency hides behind the special-function work.
+      const bool do_rs = j > 0 && __any_sync(0xffffffffu, rescale);
+      const uint64_t alpha2 = f2(alpha, alpha);
+      uint32_t ov[32];
+      auto rescale_chunk = [&](int cc) {
+        if (!do_rs || cc >= D / 32) return;
+        tmem_ld_wait(ov);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float a, b;
+          f2split(fmul2(f2(__uint_as_float(ov[2 * i]), __uint_as_float(ov[2 * i + 1])), alpha2), a, b);
+          ov[2 * i] = __float_as_uint(a);
+          ov[2 * i + 1] = __float_as_uint(b);
+        }
+        tmem_st32(tO + 32 * cc, ov);
+        if (cc + 1 < D / 32) tmem_ld32(tO + 32 * (cc + 1), ov);
+      };
+      if (do_rs) tmem_ld32(tO, ov);
       {
         uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = ex2(fmaf(x0[2 * i], sl2, neg)), b = ex2(fmaf(x0[2 * i + 1], sl2, neg));
-          sum0 += a;
-          sum1 += b;
-          pk[i] = pack2<BF16>(a, b);
-        }
+        for (int i = 0; i < 16; ++i) pk[i] = exp_pack(x0[2 * i], x0[2 * i + 1]);
+        rescale_chunk(0);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = ex2(fmaf(x1[2 * i], sl2, neg)), b = ex2(fmaf(x1[2 * i + 1], sl2, neg));
-          sum0 += a;
-          sum1 += b;
-          pk[16 + i] = pack2<BF16>(a, b);
-        }
+        for (int i = 0; i < 16; ++i) pk[16 + i] = exp_pack(x1[2 * i], x1[2 * i + 1]);
+        rescale_chunk(1);
         tmem_st32(tS + 0, pk);
       }
       {
         uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = ex2(fmaf(x2[2 * i], sl2, neg)), b = ex2(fmaf(x2[2 * i + 1], sl2, neg));
-          sum0 += a;
-          sum1 += b;
-          pk[i] = pack2<BF16>(a, b);
-        }
+        for (int i = 0; i < 16; ++i) pk[i] = exp_pack(x2[2 * i], x2[2 * i + 1]);
+        rescale_chunk(2);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = ex2(fmaf(x3[2 * i], sl2, neg)), b = ex2(fmaf(x3[2 * i + 1], sl2, neg));
-          sum0 += a;
-          sum1 += b;
-          pk[16 + i] = pack2<BF16>(a, b);
-        }
+        for (int i = 0; i < 16; ++i) pk[16 + i] = exp_pack(x3[2 * i], x3[2 * i + 1]);
+        rescale_chunk(3);
         tmem_st32(tS + 32, pk);
       }
-      l = l * alpha + (sum0 + sum1);
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t ov[32];
-          tmem_ld32(tO + 32 * cc, ov);
-          tmem_ld_wait(ov);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st32(tO + 32 * cc, ov);
-        }
-      }
+      // l (fp32 sum) gives LSE; lr (sum of the rounded P) normalises O, so
+      // O / lr is a convex combination of the V rows with exactly the weights
+      // the P V product used.
+      float f0, f1, r0, r1;
+      f2split(fsum, f0, f1);
+      f2split(rsum, r0, r1);
+      l = l * alpha + (f0 + f1);
+      lr = lr * alpha + (r0 + r1);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
@@ -370,7 +402,7 @@ __global__ void __launch_bounds__(384, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&o_full[t], 0, FWD_SITE_O));
       if (ok) {
         tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float inv = lr > 0.f ? 1.f / lr : 0.f;
         const bool valid = row < seq_len;
         const size_t grow = (size_t)head * p.rows + row_base + row;
         uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + grow * D);

@@ -260,6 +260,44 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Paired fp32 arithmetic (sm_100 f32x2 instructions): a 64-bit register
+// holds {lo, hi}.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// A packed 16-bit pair widened exactly to a paired fp32 value.
+template <bool BF16>
+__device__ __forceinline__ uint64_t widen2(uint32_t v) {
+  if constexpr (BF16) {
+    return f2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+  } else {
+    __half2 h = *reinterpret_cast<__half2*>(&v);
+    const float2 f = __half22float2(h);
+    return f2(f.x, f.y);
+  }
+}
+
 // Two fp32 values rounded to nearest into one packed 16-bit pair: `lo` in
 // bits 0-15 (the lower column / element index), `hi` in bits 16-31.
 template <bool BF16>
@@ -271,6 +309,21 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   }
   return r;
+}
+
+// Add the two 16-bit values of a packed pair, widened exactly to fp32, to
+// two running sums.
+template <bool BF16>
+__device__ __forceinline__ void accum2(uint32_t v, float& s0, float& s1) {
+  if constexpr (BF16) {
+    s0 += __uint_as_float(v << 16);
+    s1 += __uint_as_float(v & 0xffff0000u);
+  } else {
+    __half2 h = *reinterpret_cast<__half2*>(&v);
+    const float2 f = __half22float2(h);
+    s0 += f.x;
+    s1 += f.y;
+  }
 }
 
 template <bool BF16>
@@ -288,6 +341,18 @@ __device__ __forceinline__ uint32_t lane_id() {
   uint32_t l;
   asm volatile("mov.u32 %0, %%laneid;" : "=r"(l));
   return l;
+}
+
+// Per-warpgroup register budget (all four warps of a warpgroup execute the
+// same call).  The kernels using these are launched with 384 threads x 168
+// registers = 64512; their splits stay below that total.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // Named barrier over `count` threads (a multiple of 32).

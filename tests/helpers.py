@@ -20,16 +20,34 @@ def f64(t) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
+def _round_like(x: np.ndarray, dtype) -> np.ndarray:
+    return torch.from_numpy(x).to(dtype).double().numpy()
+
+
 def check_o(o_gpu, o_ref, what=""):
+    """O within the stated bounds of the fp64 oracle.
+
+    O is returned in the input dtype, so an element can never be closer to
+    the oracle than the oracle rounded to that dtype: for bf16 that half-ulp
+    is 2^-8 |O| and exceeds 1e-2 once |O| >= 4.  Such elements (and only
+    those) are held to the 1e-2 bound against the oracle rounded to the
+    output dtype; the raw max-abs error is still reported in the message.
+    """
+    dtype = o_gpu.dtype if isinstance(o_gpu, torch.Tensor) else torch.float64
     o_gpu, o_ref = f64(o_gpu), f64(o_ref)
     assert np.isfinite(o_gpu).all(), f"{what}: non-finite O"
-    err = np.abs(o_gpu - o_ref)
-    emax, emean = err.max(), err.mean()
+    raw = np.abs(o_gpu - o_ref)
+    err = raw
+    if raw.max() > O_MAX and dtype in (torch.bfloat16, torch.float16):
+        rounding = np.abs(_round_like(o_ref, dtype) - o_ref)
+        beyond = rounding > O_MAX  # the dtype cannot represent the oracle to 1e-2 here
+        err = np.where(beyond, np.abs(o_gpu - _round_like(o_ref, dtype)), raw)
+    emax, emean = err.max(), raw.mean()
     if emax > O_MAX or emean > O_MEAN:
         idx = np.unravel_index(err.argmax(), err.shape)
-        raise AssertionError(f"{what}: O max-abs {emax:.3e} (limit {O_MAX}) mean-abs {emean:.3e} "
-                             f"(limit {O_MEAN}); worst at {idx}: gpu {o_gpu[idx]:.5f} ref {o_ref[idx]:.5f}")
-    return emax, emean
+        raise AssertionError(f"{what}: O max-abs {emax:.3e} (raw {raw.max():.3e}, limit {O_MAX}) mean-abs "
+                             f"{emean:.3e} (limit {O_MEAN}); worst at {idx}: gpu {o_gpu[idx]:.5f} ref {o_ref[idx]:.5f}")
+    return raw.max(), emean
 
 
 def check_lse(l_gpu, l_ref, what=""):
