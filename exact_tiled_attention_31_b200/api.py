@@ -27,7 +27,10 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = ran
 FA_BF16, FA_FP16 = 0, 1
 
 EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
-           "fa_bwd_finish", "fa_status_string", "fa_check_device_error", "fa_launch_count")
+           "fa_bwd_finish", "fa_bwd_noalloc", "fa_status_string", "fa_check_device_error", "fa_launch_count")
+
+# Fixed scratch size of fa_bwd_noalloc (FA_BWD_NOALLOC_SCRATCH_BYTES in include/fa.h).
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 _lib = None
 
@@ -63,6 +66,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_bwd_main.restype = i
     lib.fa_bwd_finish.argtypes = [vp, i, i, i, i, f, i, vp, sz, vp]
     lib.fa_bwd_finish.restype = i
+    lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+    lib.fa_bwd_noalloc.restype = i
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_check_device_error.argtypes = [vp]
@@ -106,6 +111,12 @@ def fa_bwd_main(q, k, v, dO, dk, dv, B, H, S, D, scale, causal, dt, deterministi
 
 def fa_bwd_finish(dq, B, H, S, D, scale, dt, workspace, workspace_bytes, stream) -> int:
     return load_library().fa_bwd_finish(dq, B, H, S, D, scale, dt, workspace, workspace_bytes, stream)
+
+
+def fa_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, causal, dt, deterministic,
+                   stream) -> int:
+    return load_library().fa_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, int(causal), dt,
+                                         int(deterministic), stream)
 
 
 def fa_status_string(status: int) -> str:
@@ -200,6 +211,22 @@ def backward(q, k, v, o, do, lse, causal: bool, scale: float | None = None, dete
                 workspace.data_ptr(), workspace.numel(), _stream(stream))
     if st != FA_OK:
         raise FAError(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def backward_noalloc(q, k, v, o, do, lse, dq, dk, dv, causal: bool, scale: float | None = None,
+                     deterministic: bool = False, stream=None):
+    """Backward into caller-provided dq, dk, dv with no allocation at all:
+    the library's fixed device scratch replaces the workspace (for callers
+    that must not allocate device memory; sizes beyond the scratch raise)."""
+    B, H, S, D = q.shape
+    _check((q, k, v, o, do, dq, dk, dv), q.shape)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    st = fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, S, D, scale, causal, _dt(q),
+                        deterministic, _stream(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd_noalloc")
     return dq, dk, dv
 
 

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <initializer_list>
+#include <mutex>
 
 #include "../../include/fa.h"
 #include "fa_bwd.cuh"
@@ -234,6 +235,29 @@ bool ptrs_ok(std::initializer_list<const void*> ps) {
   return true;
 }
 
+// ---------------------------------------------------------------- allocation-free backward
+// Scratch of fa_bwd_noalloc: a fixed array in device memory, created when
+// the library's module is loaded on a device and held until the process
+// exits.  Host code only sees a host-side stand-in under this name; the
+// device address is looked up once per device below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up on
+// the first call per device (with that device current) and cached.
+void* noalloc_scratch() {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -329,6 +353,24 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                   stream);
   if (c != FA_OK) return c;
   return fa_bwd_finish(dq, B, H, S, D, scale, dt, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int D, float scale,
+                         int causal, fa_dtype dt, int deterministic, void* stream) {
+  if (B < 0 || H < 0 || S < 0) return FA_ERR_INVALID_ARG;
+  if (dt != FA_BF16 && dt != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || S == 0) return FA_OK;
+  if ((long long)B * H > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  if (!ptrs_ok({q, k, v, o, dO, lse, dq, dk, dv})) return FA_ERR_INVALID_ARG;
+  // sizes whose scratch does not fit the fixed array are refused up front
+  if (fa_bwd_workspace_size(B, H, S, D) > (size_t)FA_BWD_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
+  void* scratch = noalloc_scratch();
+  if (!scratch) return FA_ERR_CUDA;
+  return fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, causal, dt, deterministic, scratch,
+                (size_t)FA_BWD_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 const char* fa_status_string(fa_status s) {

@@ -138,6 +138,37 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* d
 fa_status fa_bwd_finish(void* dq, int B, int H, int S, int D, float scale, fa_dtype dt,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Backward pass that allocates nothing and takes no workspace.
+ *
+ * Some callers cannot call cudaMalloc: code that runs inside a device memory
+ * allocator's own hooks (a nested allocation would re-enter it), processes
+ * whose device memory is planned up front and must not grow while they run,
+ * and latency-critical loops where an allocation may stall on the device.
+ * For them, fa_bwd_noalloc computes exactly what fa_bwd computes (same
+ * arguments, same results, same deterministic option) but keeps its scratch
+ * (the fp32 dQ accumulator, the D_i and LSE rows, the ordering counters) in
+ * one fixed array of FA_BWD_NOALLOC_SCRATCH_BYTES bytes that lives in device
+ * memory from the moment the library is loaded on a device until the
+ * process exits.  The caller still provides every input and output.
+ *   - Sizes with fa_bwd_workspace_size(B, H, S, D) > FA_BWD_NOALLOC_SCRATCH_BYTES
+ *     are refused with FA_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on each device looks up that array's device address
+ *     (with the device current) and caches it; make that first call before
+ *     any stream capture.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents; each call clears what must start at zero itself.
+ *     Calls whose kernels overlap on the GPU (different streams without
+ *     ordering between them) race on the array: serialise them.
+ *   - It never calls cudaMalloc, cudaFree or any allocating library routine.
+ * The pages describe no such variant; it exists for the callers above.
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const float* lse, void* dq, void* dk, void* dv,
+                         int B, int H, int S, int D, float scale, int causal, fa_dtype dt,
+                         int deterministic, void* stream);
+
 /* A static, human-readable name for a status code. */
 const char* fa_status_string(fa_status s);
 
