@@ -201,9 +201,9 @@ fa_status launch_bwd_main(const void* q, const void* k, const void* v, const voi
                          : set_smem<fa::bwd_main_kernel<D, BF16, false>>(C::SMEM);
   if (e != cudaSuccess) return FA_ERR_CUDA;
   if (causal)
-    fa::bwd_main_kernel<D, BF16, true><<<(unsigned)grid, 384, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, p);
+    fa::bwd_main_kernel<D, BF16, true><<<(unsigned)grid, 512, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, p);
   else
-    fa::bwd_main_kernel<D, BF16, false><<<(unsigned)grid, 384, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, p);
+    fa::bwd_main_kernel<D, BF16, false><<<(unsigned)grid, 512, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, p);
   g_launches.fetch_add(1);
   return from_cuda(cudaGetLastError());
 }

@@ -15,7 +15,7 @@
 //   bwd_pre   D_i = dO_i . O_i (fp32, warp-shuffle reduction), LSE_i*log2(e)
 //             into a 128-row-padded copy, zero the fp32 dQ accumulator and
 //             the ordering counters.
-//   bwd_main  one CTA per 128-row key/value tile j of one head (384 threads):
+//   bwd_main  one CTA per 128-row key/value tile j of one head (512 threads):
 //               warp 0     TMA producer: K_j, V_j once; then Q_i (+ the padded
 //                          LSE/D rows of tile i) into a 2-slot ring and dO_i
 //                          into its own slot.
@@ -191,7 +191,7 @@ __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
 // bwd_main
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
@@ -235,8 +235,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(do_empty, 1);
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(ds_full, 128);
+    mbar_init(p_full, 256);
+    mbar_init(ds_full, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
     mbar_init(dkv_full, 1);
@@ -253,6 +253,11 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  // register split over 512 threads launched with 128 each (65536):
+  // 128 x 56 (warps 0-3) + 256 x 152 (P/dS) + 128 x 144 (dQ) = 64512.
+  // Each warpgroup changes its budget inside its own branch.
+  if (warp < 4) {
+  regs_dec<56>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -295,78 +300,95 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t ID_KK = make_idesc(128, 128, BF16, false, false);  // dP^T, S^T
-      constexpr uint32_t ID_TS = make_idesc(128, D, BF16, false, true);     // dV, dK
-      constexpr uint32_t ID_DQ = make_idesc(128, D, BF16, true, true);      // dQ
-      const uint32_t sk = smem_addr(smem + C::K_OFF), sv = smem_addr(smem + C::V_OFF);
-      const uint32_t sq = smem_addr(smem + C::Q_OFF), sdo = smem_addr(smem + C::DO_OFF);
-      const uint32_t sds = smem_addr(smem + C::DS_OFF);
-      // X^T = A_kv B_q^T with both operands K-major (X = S or dP)
-      auto kk_product = [&](uint32_t d_col, uint32_t a, uint32_t b) {
+    // Converged warp, one elected lane issues; descriptors formed once and
+    // offset by constants inside fully unrolled groups of 8 products.
+    const uint32_t e = elect_one();
+    constexpr uint32_t ID_KK = make_idesc(128, 128, BF16, false, false);  // dP^T, S^T
+    constexpr uint32_t ID_TS = make_idesc(128, D, BF16, false, true);     // dV, dK
+    constexpr uint32_t ID_DQ = make_idesc(128, D, BF16, true, true);      // dQ
+    const uint64_t kK = make_sdesc(smem_addr(smem + C::K_OFF), 16, 1024);       // K as A (K-major)
+    const uint64_t kMN = make_sdesc(smem_addr(smem + C::K_OFF), C::CHUNK, 1024);  // K as B of dQ (MN-major)
+    const uint64_t vK = make_sdesc(smem_addr(smem + C::V_OFF), 16, 1024);
+    const uint64_t qK = make_sdesc(smem_addr(smem + C::Q_OFF), 16, 1024);       // Q slot 0 as B of S^T
+    const uint64_t qMN = make_sdesc(smem_addr(smem + C::Q_OFF), C::CHUNK, 1024);  // Q slot 0 as B of dK
+    const uint64_t doK = make_sdesc(smem_addr(smem + C::DO_OFF), 16, 1024);
+    const uint64_t doMN = make_sdesc(smem_addr(smem + C::DO_OFF), C::CHUNK, 1024);
+    const uint64_t dsMN = make_sdesc(smem_addr(smem + C::DS_OFF), C::CHUNK, 1024);
+    // X^T = A_kv B_q^T with both operands K-major (X = S or dP)
+    auto kk_product = [&](uint32_t d_col, uint64_t a, uint64_t b) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + d_col, make_sdesc(a + off, 16, 1024), make_sdesc(b + off, 16, 1024), ID_KK, kk > 0);
-        }
-      };
-      bool ok = mbar_wait(kv_full, 0, BWD_SITE_KV) && mbar_wait(&q_full[0], 0, BWD_SITE_Q) &&
-                mbar_wait(do_full, 0, BWD_SITE_DO);
-      if (ok) {
-        kk_product(C::TM_A, sk, sq);  // S^T(0)
-        mma_commit(s_full);
-        kk_product(C::TM_B, sv, sdo);  // dP^T(0)
-        mma_commit(dp_full);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+        mma_ss_e(tmem + d_col, desc_add(a, off), desc_add(b, off), ID_KK, kk > 0 ? 1u : 0u, e);
       }
-      for (int st = 0; st < n_steps && ok; ++st) {
-        const int qs = st & 1;
-        // dV += P^T dO_i
-        if (!(ok = mbar_wait(p_full, st & 1, BWD_SITE_P))) break;
-        tc_fence_after();
+    };
+    // acc += A(TMEM, 16-bit pairs) * B (MN-major), K = 128 queries.  Queries
+    // 0-63 sit in the first 32 columns of the A region, queries 64-127 in
+    // columns 64-95 (each half is written by the warpgroup that read those
+    // score columns).
+    auto ts_product = [&](uint32_t d_col, uint32_t a_col, uint64_t b, uint32_t acc) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + C::TM_DV, tmem + C::TM_A + kk * 8, make_sdesc(sdo + kk * 2048, C::CHUNK, 1024), ID_TS,
-                 (st > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(do_empty);
-        // S^T(i+1) into A (P^T(i) has been read by the products above)
-        const bool more = st + 1 < n_steps;
-        if (more) {
-          if (!(ok = mbar_wait(&q_full[qs ^ 1], ((st + 1) >> 1) & 1, BWD_SITE_Q))) break;
-          kk_product(C::TM_A, sk, sq + (qs ^ 1) * C::TILE);
-          mma_commit(s_full);
-        }
-        // dK += dS^T Q_i
-        if (!(ok = mbar_wait(ds_full, st & 1, BWD_SITE_DS))) break;
-        tc_fence_after();
-        const uint32_t qa = sq + qs * C::TILE;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + C::TM_DK, tmem + C::TM_B + kk * 8, make_sdesc(qa + kk * 2048, C::CHUNK, 1024), ID_TS,
-                 (st > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&q_empty[qs]);
-        // dQ_i = dS K_j into B  (A = dS MN-major in smem, B = K MN-major)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + C::TM_B, make_sdesc(sds + kk * 2048, C::CHUNK, 1024),
-                 make_sdesc(sk + kk * 2048, C::CHUNK, 1024), ID_DQ, kk > 0);
-        mma_commit(dq_full);
-        // dP^T(i+1) into B once dQ_i has been drained
-        if (more) {
-          if (!(ok = mbar_wait(dq_empty, st & 1, BWD_SITE_DQE))) break;
-          if (!(ok = mbar_wait(do_full, (st + 1) & 1, BWD_SITE_DO))) break;
-          tc_fence_after();
-          kk_product(C::TM_B, sv, sdo);
-          mma_commit(dp_full);
-        }
-      }
-      mma_commit(dkv_full);
-      mma_commit(drain);
-      mbar_wait(drain, 0, BWD_SITE_DRAIN);
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts_e(tmem + d_col, tmem + a_col + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), desc_add(b, kk * 2048), ID_TS,
+                 kk > 0 ? 1u : acc, e);
+    };
+    bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0, BWD_SITE_KV) && mbar_wait(&q_full[0], 0, BWD_SITE_Q) &&
+                                          mbar_wait(do_full, 0, BWD_SITE_DO));
+    if (ok) {
+      tc_fence_after();
+      kk_product(C::TM_A, kK, qK);  // S^T(0)
+      mma_commit_e(s_full, e);
+      kk_product(C::TM_B, vK, doK);  // dP^T(0)
+      mma_commit_e(dp_full, e);
     }
+    for (int st = 0; st < n_steps && ok; ++st) {
+      const int qs = st & 1;
+      const uint32_t acc = st > 0 ? 1u : 0u;
+      // dV += P^T dO_i
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_full, st & 1, BWD_SITE_P)))) break;
+      tc_fence_after();
+      ts_product(C::TM_DV, C::TM_A, doMN, acc);
+      mma_commit_e(do_empty, e);
+      // S^T(i+1) into A (P^T(i) has been read by the products above)
+      const bool more = st + 1 < n_steps;
+      if (more) {
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&q_full[qs ^ 1], ((st + 1) >> 1) & 1, BWD_SITE_Q)))) break;
+        tc_fence_after();
+        kk_product(C::TM_A, kK, desc_add(qK, (qs ^ 1) * C::TILE));
+        mma_commit_e(s_full, e);
+      }
+      // dK += dS^T Q_i
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_full, st & 1, BWD_SITE_DS)))) break;
+      tc_fence_after();
+      ts_product(C::TM_DK, C::TM_B, desc_add(qMN, qs * C::TILE), acc);
+      mma_commit_e(&q_empty[qs], e);
+      // dQ_i = dS K_j into B  (A = dS MN-major in smem, B = K MN-major)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ss_e(tmem + C::TM_B, desc_add(dsMN, kk * 2048), desc_add(kMN, kk * 2048), ID_DQ, kk > 0 ? 1u : 0u, e);
+      mma_commit_e(dq_full, e);
+      // dP^T(i+1) into B once dQ_i has been drained
+      if (more) {
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_empty, st & 1, BWD_SITE_DQE)))) break;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(do_full, (st + 1) & 1, BWD_SITE_DO)))) break;
+        tc_fence_after();
+        kk_product(C::TM_B, vK, doK);
+        mma_commit_e(dp_full, e);
+      }
+    }
+    mma_commit_e(dkv_full, e);
+    mma_commit_e(drain, e);
+    mbar_wait(drain, 0, BWD_SITE_DRAIN);
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ P / dS (one thread per key row)
-    const int r = threadIdx.x - 128;
+  }
+  } else if (warp < 12) {
+    regs_inc<152>();
+    // ------------------------------------------------------------ P / dS
+    // One thread per key row and half of the 128 query columns: warps 4-7
+    // take queries 0-63, warps 8-11 queries 64-127.  P and dS are
+    // elementwise given LSE and D_i, so the halves never exchange data.
+    const int half = (warp - 4) >> 2;
+    const int r = (threadIdx.x - 128) & 127;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tA = tmem + lane_off + C::TM_A, tB = tmem + lane_off + C::TM_B;
     const int kv = kv_row0 + r;
@@ -385,16 +407,17 @@ __global__ void __launch_bounds__(384, 1)
       const float* dlt = lse2 + 128;
       // visible queries of this key row in tile i: q >= kv under the causal mask
       const int qlo = (CAUSAL && i == j) ? r : 0;
-      // ---- P phase
-      uint32_t pk[64];
+      // ---- P phase (score columns 64*half .. +63)
+      uint32_t pk[32];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < 2; ++ch) {
+        const int c0 = 64 * half + 32 * ch;
         uint32_t sv[32];
-        tmem_ld32(tA + 32 * ch, sv);
+        tmem_ld32(tA + c0, sv);
         tmem_ld_wait(sv);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int c = 32 * ch + 2 * e;
+          const int c = c0 + 2 * e;
           float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -lse2[c]));
           float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -lse2[c + 1]));
           if (c < qlo || !kv_valid) p0 = 0.f;
@@ -402,12 +425,9 @@ __global__ void __launch_bounds__(384, 1)
           pk[16 * ch + e] = pack2<BF16>(p0, p1);
         }
       }
-      {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-        tmem_st32(tA, lo);
-        tmem_st32(tA + 32, hi);
-      }
+      // P^T pairs go to columns [64*half, 64*half + 32) of A (inside this
+      // half's own score columns, already read)
+      tmem_st32(tA + 64 * half, pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
@@ -415,28 +435,31 @@ __global__ void __launch_bounds__(384, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, st & 1, BWD_SITE_DP));
       if (!ok) break;
       tc_fence_after();
+      uint32_t dd[32];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < 2; ++ch) {
+        const int c0 = 64 * half + 32 * ch;
         uint32_t dv[32];
-        tmem_ld32(tB + 32 * ch, dv);
+        tmem_ld32(tB + c0, dv);
         tmem_ld_wait(dv);
-        uint32_t dd[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int c = 32 * ch + 2 * e;
+          const int c = c0 + 2 * e;
           const float2 pp = unpack2<BF16>(pk[16 * ch + e]);
-          dd[e] = pack2<BF16>(pp.x * (__uint_as_float(dv[2 * e]) - dlt[c]),
-                              pp.y * (__uint_as_float(dv[2 * e + 1]) - dlt[c + 1]));
+          dd[16 * ch + e] = pack2<BF16>(pp.x * (__uint_as_float(dv[2 * e]) - dlt[c]),
+                                        pp.y * (__uint_as_float(dv[2 * e + 1]) - dlt[c + 1]));
         }
-        tmem_st16(tB + 16 * ch, dd);
-        // dS row r (key) holds 32 query columns of chunk ch: MN-major A operand
-        // of dQ = dS K, i.e. [key][query] with queries contiguous, 128-B swizzled.
-        const uint32_t base = (ch >> 1) * C::CHUNK + r * 128 + (ch & 1) * 64;
+        // dS row r (key), 32 query columns: MN-major A operand of dQ = dS K,
+        // [key][query] with queries contiguous, 64-query chunk = half, 128-B swizzled
+        const uint32_t base = half * C::CHUNK + r * 128 + ch * 64;
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4)
           *reinterpret_cast<uint4*>(ds_smem + swz128(base + v4 * 16)) =
-              make_uint4(dd[4 * v4], dd[4 * v4 + 1], dd[4 * v4 + 2], dd[4 * v4 + 3]);
+              make_uint4(dd[16 * ch + 4 * v4], dd[16 * ch + 4 * v4 + 1], dd[16 * ch + 4 * v4 + 2],
+                         dd[16 * ch + 4 * v4 + 3]);
       }
+      // dS^T pairs to columns [64*half, 64*half + 32) of B (dP columns already read)
+      tmem_st32(tB + 64 * half, dd);
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
@@ -447,8 +470,8 @@ __global__ void __launch_bounds__(384, 1)
     if (ok) {
       tc_fence_after();
       const size_t grow = ((size_t)head * p.S + kv) * D;
-#pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
+      {
+        const int which = half;  // half 0 writes dV, half 1 writes scale * dK
         uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(which ? p.dk : p.dv) + grow);
         const float mul = which ? p.scale : 1.f;
         const uint32_t col = which ? C::TM_DK : C::TM_DV;
@@ -469,10 +492,11 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
     }
-  } else if (warp >= 8) {
+  } else {
+    regs_inc<144>();
     // ------------------------------------------------------------ dQ (one thread per query row)
-    const int c = threadIdx.x - 256;                 // query row within the tile = TMEM lane
-    const int wq = warp - 8;                         // this warp's 32 rows: 32*wq ..
+    const int c = threadIdx.x - 384;                 // query row within the tile = TMEM lane
+    const int wq = warp - 12;                        // this warp's 32 rows: 32*wq ..
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     uint8_t* stg = smem + C::STG_OFF + wq * 4096;    // 32 rows x 128 B, 128-B swizzled
     if (!p.deterministic && lane == 0) tma_prefetch_desc(&tm_dq);

@@ -192,88 +192,94 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC_QK = make_idesc(128, 128, BF16, false, false);
-      constexpr uint32_t IDESC_PV = make_idesc(128, D, BF16, false, true);
-      uint32_t use = 0;
-      bool ok = mbar_wait(&q_full[0], 0, FWD_SITE_Q);
-      auto next_slot = [&](uint32_t& slot) {
-        slot = use % C::NSLOT;
-        if (ok) ok = mbar_wait(&kv_full[slot], (use / C::NSLOT) & 1, FWD_SITE_KV);
-        ++use;
-      };
-      // S_t = Q_t K^T: M = 128 query rows, N = 128 keys, K = D (both K-major)
-      auto qk = [&](int t, uint32_t kslot) {
-        const uint32_t qa = sq + t * C::TILE, ka = skv + kslot * C::TILE;
+    // The whole warp runs this converged; one elected lane issues.  Operand
+    // descriptors are formed once and offset by constants inside each fully
+    // unrolled group of products.
+    const uint32_t e = elect_one();
+    constexpr uint32_t IDESC_QK = make_idesc(128, 128, BF16, false, false);
+    constexpr uint32_t IDESC_PV = make_idesc(128, D, BF16, false, true);
+    const uint64_t dq_base = make_sdesc(sq, 16, 1024);         // Q tile 0, K-major
+    const uint64_t dk_base = make_sdesc(skv, 16, 1024);        // K/V slot 0 as K (K-major)
+    const uint64_t dv_base = make_sdesc(skv, C::CHUNK, 1024);  // K/V slot 0 as V (MN-major)
+    uint32_t use = 0;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&q_full[0], 0, FWD_SITE_Q));
+    auto next_slot = [&](uint32_t& slot) {
+      slot = use % C::NSLOT;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[slot], (use / C::NSLOT) & 1, FWD_SITE_KV));
+      ++use;
+    };
+    // S_t = Q_t K^T: M = 128 query rows, N = 128 keys, K = D (both K-major)
+    auto qk = [&](int t, uint32_t kslot) {
+      const uint64_t a = desc_add(dq_base, t * C::TILE), b = desc_add(dk_base, kslot * C::TILE);
+      const uint32_t d = tmem + C::TM_S + 128 * t;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + C::TM_S + 128 * t, make_sdesc(qa + off, 16, 1024), make_sdesc(ka + off, 16, 1024),
-                 IDESC_QK, kk > 0);
-        }
-      };
-      // O_t += P_t V: M = 128, N = D, K = 128 keys; P from TMEM, V MN-major
-      auto pv = [&](int t, uint32_t vslot, bool acc) {
-        const uint32_t va = skv + vslot * C::TILE;
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+        mma_ss_e(d, desc_add(a, off), desc_add(b, off), IDESC_QK, kk > 0 ? 1u : 0u, e);
+      }
+    };
+    // O_t += P_t V: M = 128, N = D, K = 128 keys; P from TMEM, V MN-major
+    auto pv = [&](int t, uint32_t vslot, uint32_t acc) {
+      const uint64_t b = desc_add(dv_base, vslot * C::TILE);
+      const uint32_t d = tmem + C::TM_O + D * t, pa = tmem + C::TM_S + 128 * t;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + C::TM_O + D * t, tmem + C::TM_S + 128 * t + kk * 8, make_sdesc(va + kk * 2048, C::CHUNK, 1024),
-                 IDESC_PV, (acc || kk > 0) ? 1u : 0u);
-      };
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts_e(d, pa + kk * 8, desc_add(b, kk * 2048), IDESC_PV, kk > 0 ? 1u : acc, e);
+    };
 
-      uint32_t ks = 0;
-      next_slot(ks);
-      if (ok) {
-        qk(0, ks);
-        mma_commit(&s_full[0]);
-        if (has_t1) {
-          ok = mbar_wait(&q_full[1], 0, FWD_SITE_Q);
-          if (ok) {
-            qk(1, ks);
-            mma_commit(&s_full[1]);
-          }
-        }
-        mma_commit(&kv_empty[ks]);
-      }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        uint32_t vs = 0;
-        next_slot(vs);
-        if (!ok) break;
-        if (j < n0) {
-          if (!(ok = mbar_wait(&p_full[0], j & 1, FWD_SITE_P))) break;
-          tc_fence_after();
-          pv(0, vs, j > 0);
-          if (j == n0 - 1) mma_commit(&o_full[0]);
-        }
-        const bool more = j + 1 < n_kv;
-        uint32_t ks2 = 0;
-        if (more) {
-          next_slot(ks2);
-          if (!ok) break;
-          if (j + 1 < n0) {
-            qk(0, ks2);
-            mma_commit(&s_full[0]);
-          }
-        }
-        if (j < n1) {
-          if (!(ok = mbar_wait(&p_full[1], j & 1, FWD_SITE_P))) break;
-          tc_fence_after();
-          pv(1, vs, j > 0);
-          if (j == n1 - 1) mma_commit(&o_full[1]);
-        }
-        mma_commit(&kv_empty[vs]);
-        if (more) {
-          if (j + 1 < n1) {
-            qk(1, ks2);
-            mma_commit(&s_full[1]);
-          }
-          mma_commit(&kv_empty[ks2]);
+    uint32_t ks = 0;
+    next_slot(ks);
+    if (ok) {
+      tc_fence_after();
+      qk(0, ks);
+      mma_commit_e(&s_full[0], e);
+      if (has_t1) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&q_full[1], 0, FWD_SITE_Q));
+        if (ok) {
+          qk(1, ks);
+          mma_commit_e(&s_full[1], e);
         }
       }
-      // every product issued above has finished before TMEM is released
-      mma_commit(drain);
-      mbar_wait(drain, 0, FWD_SITE_DRAIN);
+      mma_commit_e(&kv_empty[ks], e);
     }
+    for (int j = 0; j < n_kv && ok; ++j) {
+      uint32_t vs = 0;
+      next_slot(vs);
+      if (!ok) break;
+      if (j < n0) {
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&p_full[0], j & 1, FWD_SITE_P)))) break;
+        tc_fence_after();
+        pv(0, vs, j > 0 ? 1u : 0u);
+        if (j == n0 - 1) mma_commit_e(&o_full[0], e);
+      }
+      const bool more = j + 1 < n_kv;
+      uint32_t ks2 = 0;
+      if (more) {
+        next_slot(ks2);
+        if (!ok) break;
+        if (j + 1 < n0) {
+          qk(0, ks2);
+          mma_commit_e(&s_full[0], e);
+        }
+      }
+      if (j < n1) {
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&p_full[1], j & 1, FWD_SITE_P)))) break;
+        tc_fence_after();
+        pv(1, vs, j > 0 ? 1u : 0u);
+        if (j == n1 - 1) mma_commit_e(&o_full[1], e);
+      }
+      mma_commit_e(&kv_empty[vs], e);
+      if (more) {
+        if (j + 1 < n1) {
+          qk(1, ks2);
+          mma_commit_e(&s_full[1], e);
+        }
+        mma_commit_e(&kv_empty[ks2], e);
+      }
+    }
+    // every product issued above has finished before TMEM is released
+    mma_commit_e(drain, e);
+    mbar_wait(drain, 0, FWD_SITE_DRAIN);
     __syncwarp();
   }
   } else {
