@@ -58,8 +58,8 @@ struct FwdCfg {
   static constexpr uint32_t Q_OFF = 0;
   static constexpr uint32_t KV_OFF = 2 * TILE;
   static constexpr uint32_t BAR_OFF = KV_OFF + NSLOT * TILE;
-  // q_full[2] kv_full[NSLOT] kv_empty[NSLOT] s_full[2] p_full[2] o_full[2] drain
-  static constexpr int NBAR = 2 + 2 * NSLOT + 7;
+  // q_full[2] kv_full[NSLOT] kv_empty[NSLOT] s_full[2] p_half[4] o_full[2] drain
+  static constexpr int NBAR = 2 + 2 * NSLOT + 9;
   static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;  // + alignment slack
   static constexpr uint32_t TM_S = 0, TM_O = 256;
   static constexpr int THREADS = 384;
@@ -116,8 +116,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* kv_full = bars + 2;
   uint64_t* kv_empty = kv_full + C::NSLOT;
   uint64_t* s_full = kv_empty + C::NSLOT;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_full = p_full + 2;
+  uint64_t* p_half = s_full + 2;  // [2 * tile + half]: P keys 0-63 / 64-127 written
+  uint64_t* o_full = p_half + 4;
   uint64_t* drain = o_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBAR);
 
@@ -128,7 +128,8 @@ __global__ void __launch_bounds__(384, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_half[2 * i], 128);
+      mbar_init(&p_half[2 * i + 1], 128);
       mbar_init(&o_full[i], 1);
     }
     for (int i = 0; i < C::NSLOT; ++i) {
@@ -218,13 +219,22 @@ __global__ void __launch_bounds__(384, 1)
         mma_ss_e(d, desc_add(a, off), desc_add(b, off), IDESC_QK, kk > 0 ? 1u : 0u, e);
       }
     };
-    // O_t += P_t V: M = 128, N = D, K = 128 keys; P from TMEM, V MN-major
-    auto pv = [&](int t, uint32_t vslot, uint32_t acc) {
+    // O_t += P_t V: M = 128, N = D, K = 128 keys; P from TMEM, V MN-major.
+    // Keys 0-63 (k-steps 0-3) once the first half of P is published, keys
+    // 64-127 once the second is.
+    auto pv = [&](int t, uint32_t vslot, uint32_t acc, int j) -> bool {
       const uint64_t b = desc_add(dv_base, vslot * C::TILE);
       const uint32_t d = tmem + C::TM_O + D * t, pa = tmem + C::TM_S + 128 * t;
+      if (!__all_sync(0xffffffffu, mbar_wait(&p_half[2 * t], j & 1, FWD_SITE_P))) return false;
+      tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
+      for (int kk = 0; kk < 4; ++kk)
         mma_ts_e(d, pa + kk * 8, desc_add(b, kk * 2048), IDESC_PV, kk > 0 ? 1u : acc, e);
+      if (!__all_sync(0xffffffffu, mbar_wait(&p_half[2 * t + 1], j & 1, FWD_SITE_P))) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 4; kk < 8; ++kk) mma_ts_e(d, pa + kk * 8, desc_add(b, kk * 2048), IDESC_PV, 1u, e);
+      return true;
     };
 
     uint32_t ks = 0;
@@ -247,9 +257,7 @@ __global__ void __launch_bounds__(384, 1)
       next_slot(vs);
       if (!ok) break;
       if (j < n0) {
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&p_full[0], j & 1, FWD_SITE_P)))) break;
-        tc_fence_after();
-        pv(0, vs, j > 0 ? 1u : 0u);
+        if (!(ok = pv(0, vs, j > 0 ? 1u : 0u, j))) break;
         if (j == n0 - 1) mma_commit_e(&o_full[0], e);
       }
       const bool more = j + 1 < n_kv;
@@ -263,9 +271,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       if (j < n1) {
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&p_full[1], j & 1, FWD_SITE_P)))) break;
-        tc_fence_after();
-        pv(1, vs, j > 0 ? 1u : 0u);
+        if (!(ok = pv(1, vs, j > 0 ? 1u : 0u, j))) break;
         if (j == n1 - 1) mma_commit_e(&o_full[1], e);
       }
       mma_commit_e(&kv_empty[vs], e);
@@ -325,9 +331,16 @@ __global__ void __launch_bounds__(384, 1)
           if (c + 96 >= limit) x3[c] = -INFINITY;
         }
       }
-      float mx = -INFINITY;
+      // row max as a tree of independent 3-input maxima
+      float mxa = -INFINITY, mxb = -INFINITY, mxc = -INFINITY, mxd = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(fmaxf(x0[c], x1[c]), fmaxf(x2[c], x3[c])));
+      for (int c = 0; c < 32; c += 2) {
+        mxa = fmax3(mxa, x0[c], x0[c + 1]);
+        mxb = fmax3(mxb, x1[c], x1[c + 1]);
+        mxc = fmax3(mxc, x2[c], x2[c + 1]);
+        mxd = fmax3(mxd, x3[c], x3[c + 1]);
+      }
+      const float mx = fmax3(mxa, mxb, fmaxf(mxc, mxd));
       // Rescale O and the running sums only when the row max actually grew
       // (by more than kRescaleLog2): every P is then <= 2^kRescaleLog2, and
       // with kRescaleLog2 = 0 the largest P of the row is exactly 1.
@@ -339,20 +352,33 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t scale2 = f2(sl2, sl2), neg2 = f2(neg, neg);
       // fsum: fp32 sum of P (for LSE); rsum: sum of P as rounded to 16 bits
       // (the weights the P V product uses, for normalising O).
-      uint64_t fsum = f2(0.f, 0.f), rsum = f2(0.f, 0.f);
-      auto exp_pack = [&](float x, float y) -> uint32_t {
-        float a, b;
-        f2split(ffma2(f2(x, y), scale2, neg2), a, b);
-        a = ex2(a);
-        b = ex2(b);
-        fsum = fadd2(fsum, f2(a, b));
+      uint64_t fsum0 = f2(0.f, 0.f), fsum1 = f2(0.f, 0.f), rsum0 = f2(0.f, 0.f), rsum1 = f2(0.f, 0.f);
+      auto finish_pair = [&](float a, float b, uint64_t& fs, uint64_t& rs) -> uint32_t {
+        fs = fadd2(fs, f2(a, b));
         const uint32_t pk = pack2<BF16>(a, b);
-        rsum = fadd2(rsum, widen2<BF16>(pk));
+        rs = fadd2(rs, widen2<BF16>(pk));
         return pk;
       };
+      // P from the special-function unit
+      auto exp_sfu = [&](float x, float y, uint64_t& fs, uint64_t& rs) -> uint32_t {
+        float a, b;
+        f2split(ffma2(f2(x, y), scale2, neg2), a, b);
+        return finish_pair(ex2(a), ex2(b), fs, rs);
+      };
+      // P from the FMA pipe (exp2_poly2): used for the last 32 columns of
+      // tiles every row of this warp sees in full, to share the exponentials
+      // between the two pipes.
+      const bool full_tile = __all_sync(0xffffffffu, limit == 128);
+      auto exp_fma = [&](float x, float y, uint64_t& fs, uint64_t& rs) -> uint32_t {
+        float a, b;
+        f2split(exp2_poly2(ffma2(f2(x, y), scale2, neg2)), a, b);
+        return finish_pair(a, b, fs, rs);
+      };
       // O_t (written by the previous P V product, complete once S_t arrived)
-      // is rescaled 32 columns at a time, each load issued one exponential
-      // chunk ahead so its latency hides behind the special-function work.
+      // is rescaled 32 columns at a time while the first half of P is made;
+      // each load is issued one step ahead so its latency hides behind the
+      // exponentials.  The first half of P (keys 0-63) is published before the
+      // second is computed, so the P V product can start on it.
       const bool do_rs = j > 0 && __any_sync(0xffffffffu, rescale);
       const uint64_t alpha2 = f2(alpha, alpha);
       uint32_t ov[32];
@@ -373,34 +399,48 @@ __global__ void __launch_bounds__(384, 1)
       {
         uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = exp_pack(x0[2 * i], x0[2 * i + 1]);
+        for (int i = 0; i < 8; ++i) pk[i] = exp_sfu(x0[2 * i], x0[2 * i + 1], fsum0, rsum0);
         rescale_chunk(0);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[16 + i] = exp_pack(x1[2 * i], x1[2 * i + 1]);
+        for (int i = 8; i < 16; ++i) pk[i] = exp_sfu(x0[2 * i], x0[2 * i + 1], fsum1, rsum1);
         rescale_chunk(1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pk[16 + i] = exp_sfu(x1[2 * i], x1[2 * i + 1], fsum0, rsum0);
+        rescale_chunk(2);
+#pragma unroll
+        for (int i = 8; i < 16; ++i) pk[16 + i] = exp_sfu(x1[2 * i], x1[2 * i + 1], fsum1, rsum1);
+        rescale_chunk(3);
         tmem_st32(tS + 0, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_half[2 * t]);
       }
       {
         uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = exp_pack(x2[2 * i], x2[2 * i + 1]);
-        rescale_chunk(2);
+        for (int i = 0; i < 16; ++i) pk[i] = exp_sfu(x2[2 * i], x2[2 * i + 1], fsum0, rsum0);
+        if (full_tile) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[16 + i] = exp_pack(x3[2 * i], x3[2 * i + 1]);
-        rescale_chunk(3);
+          for (int i = 0; i < 16; ++i) pk[16 + i] = exp_fma(x3[2 * i], x3[2 * i + 1], fsum1, rsum1);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[16 + i] = exp_sfu(x3[2 * i], x3[2 * i + 1], fsum1, rsum1);
+        }
         tmem_st32(tS + 32, pk);
       }
       // l (fp32 sum) gives LSE; lr (sum of the rounded P) normalises O, so
       // O / lr is a convex combination of the V rows with exactly the weights
       // the P V product used.
-      float f0, f1, r0, r1;
-      f2split(fsum, f0, f1);
-      f2split(rsum, r0, r1);
-      l = l * alpha + (f0 + f1);
-      lr = lr * alpha + (r0 + r1);
+      float f0, f1, f2_, f3, r0, r1, r2, r3;
+      f2split(fsum0, f0, f1);
+      f2split(fsum1, f2_, f3);
+      f2split(rsum0, r0, r1);
+      f2split(rsum1, r2, r3);
+      l = l * alpha + ((f0 + f1) + (f2_ + f3));
+      lr = lr * alpha + ((r0 + r1) + (r2 + r3));
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      mbar_arrive(&p_half[2 * t + 1]);
       m = m_new;
     }
     // ---- epilogue: O / l and LSE for the rows inside the sequence
