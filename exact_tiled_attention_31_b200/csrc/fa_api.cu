@@ -35,13 +35,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [heads, rows, D] 16-bit tensor, boxes of 128 rows x 64 columns, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int D, long long rows, long long heads, bool bf16) {
+// [heads, rows, D] 16-bit tensor, boxes of box_rows rows x 64 columns, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int D, long long rows, long long heads, bool bf16,
+              unsigned box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads};
   const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -120,9 +121,10 @@ fa_status dispatch_fwd(bool causal, bool varlen, const CUtensorMap& mq, const CU
 fa_status run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu, int heads,
                   int seqlen, long long rows, int nseq, int D, float scale, bool causal, bool bf16, bool varlen,
                   cudaStream_t st) {
+  // query tiles of 128 rows, key/value tiles of 64 rows
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, D, rows, heads, bf16) || !make_map(&mk, k, D, rows, heads, bf16) ||
-      !make_map(&mv, v, D, rows, heads, bf16))
+  if (!make_map(&mq, q, D, rows, heads, bf16, 128) || !make_map(&mk, k, D, rows, heads, bf16, 64) ||
+      !make_map(&mv, v, D, rows, heads, bf16, 64))
     return FA_ERR_CUDA;
   fa::FwdParams p;
   p.o = o;

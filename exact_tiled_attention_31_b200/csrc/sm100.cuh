@@ -427,8 +427,9 @@ __device__ __forceinline__ uint32_t lane_id() {
 }
 
 // Per-warpgroup register budget (all four warps of a warpgroup execute the
-// same call).  The kernels using these are launched with 384 threads x 168
-// registers = 64512; their splits stay below that total.
+// same call).  `inc` may only raise and `dec` only lower the count the warps
+// hold (the launch's per-thread count at first), and the new counts summed
+// over the block must stay within the registers the block was launched with.
 template <uint32_t N>
 __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
