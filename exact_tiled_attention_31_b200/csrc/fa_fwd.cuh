@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t skv = smem_addr(smem + C::KV_OFF);
 
   // register split over 512 threads launched with 128 each (65536):
-  // 128 x 40 (warps 0-3) + 256 x 184 (softmax) + 128 x 96 (correction) = 64512.
+  // 128 x 40 (warps 0-3) + 256 x 152 (softmax) + 128 x 152 (correction) = 63488.
   // Each warpgroup changes its budget inside its own branch.
   if (warp < 4) {
     regs_dec<40>();
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(512, 1)
       __syncwarp();
     }
   } else if (warp < 12) {
-    regs_inc<184>();
+    regs_inc<152>();
     // ------------------------------------------------------------ softmax
     const int t = (warp - 4) >> 2;
     const int n_t = t == 0 ? n0 : n1;
@@ -399,7 +399,7 @@ __global__ void __launch_bounds__(512, 1)
       mbar_arrive(&stats_ready[t]);
     }
   } else {
-    regs_dec<96>();
+    regs_inc<152>();
     // ------------------------------------------------------------ correction + epilogue
     const int r = 32 * (warp & 3) + (int)lane;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
@@ -418,19 +418,22 @@ __global__ void __launch_bounds__(512, 1)
           tc_fence_after();
           const uint32_t tO = tmem + lane_off + C::TM_O + D * t;
           const uint64_t alpha2 = f2(alpha, alpha);
+          // all of the row's O columns in flight at once: one load latency
+          uint32_t ov[D / 32][32];
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tO + 32 * cc, ov[cc]);
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) tmem_ld_wait(ov[cc]);
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t ov[32];
-            tmem_ld32(tO + 32 * cc, ov);
-            tmem_ld_wait(ov);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               float a, b;
-              f2split(fmul2(f2(__uint_as_float(ov[2 * i]), __uint_as_float(ov[2 * i + 1])), alpha2), a, b);
-              ov[2 * i] = __float_as_uint(a);
-              ov[2 * i + 1] = __float_as_uint(b);
+              f2split(fmul2(f2(__uint_as_float(ov[cc][2 * i]), __uint_as_float(ov[cc][2 * i + 1])), alpha2), a, b);
+              ov[cc][2 * i] = __float_as_uint(a);
+              ov[cc][2 * i + 1] = __float_as_uint(b);
             }
-            tmem_st32(tO + 32 * cc, ov);
+            tmem_st32(tO + 32 * cc, ov[cc]);
           }
           tmem_st_wait();
         }
