@@ -121,10 +121,10 @@ fa_status dispatch_fwd(bool causal, bool varlen, const CUtensorMap& mq, const CU
 fa_status run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu, int heads,
                   int seqlen, long long rows, int nseq, int D, float scale, bool causal, bool bf16, bool varlen,
                   cudaStream_t st) {
-  // query tiles of 128 rows, key/value tiles of 64 rows
+  // query and key/value tiles of 128 rows
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, D, rows, heads, bf16, 128) || !make_map(&mk, k, D, rows, heads, bf16, 64) ||
-      !make_map(&mv, v, D, rows, heads, bf16, 64))
+  if (!make_map(&mq, q, D, rows, heads, bf16, 128) || !make_map(&mk, k, D, rows, heads, bf16, 128) ||
+      !make_map(&mv, v, D, rows, heads, bf16, 128))
     return FA_ERR_CUDA;
   fa::FwdParams p;
   p.o = o;
