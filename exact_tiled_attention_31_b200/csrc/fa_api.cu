@@ -167,7 +167,7 @@ fa::BwdParams bwd_params(int heads, int S, int D, float scale, int deterministic
   p.dk = dk;
   p.dv = dv;
   p.dq_acc = reinterpret_cast<float*>(ws + w.dq_acc);
-  p.lse2 = p.lse2_w = reinterpret_cast<float*>(ws + w.lse2);
+  p.nlse2 = p.nlse2_w = reinterpret_cast<float*>(ws + w.lse2);
   p.delta = p.delta_w = reinterpret_cast<float*>(ws + w.delta);
   p.sem = reinterpret_cast<uint32_t*>(ws + w.sem);
   p.heads = heads;

@@ -12,7 +12,7 @@
 //     dQ_i  = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i
 //
 // Three launches on the caller's stream:
-//   bwd_pre   D_i = dO_i . O_i (fp32, warp-shuffle reduction), LSE_i*log2(e)
+//   bwd_pre   D_i = dO_i . O_i (fp32, warp-shuffle reduction), -LSE_i*log2(e)
 //             into a 128-row-padded copy, zero the fp32 dQ accumulator and
 //             the ordering counters.
 //   bwd_main  one CTA per 128-row key/value tile j of one head (512 threads):
@@ -56,9 +56,9 @@ struct BwdParams {
   void* dk;                // [heads, S, D]
   void* dv;                // [heads, S, D]
   float* dq_acc;           // [heads, S, D] fp32
-  const float* lse2;       // [heads, S_pad]  LSE * log2(e), +inf in padding rows
+  const float* nlse2;      // [heads, S_pad]  -LSE * log2(e), -inf in padding rows
   const float* delta;      // [heads, S_pad]  D_i, 0 in padding rows
-  float* lse2_w;           // the same two buffers, written by bwd_pre
+  float* nlse2_w;          // the same two buffers, written by bwd_pre
   float* delta_w;
   uint32_t* sem;           // [heads, n_q] ordering counters (deterministic mode)
   int heads, S, S_pad, n_q;
@@ -77,7 +77,7 @@ struct BwdCfg {
   static constexpr uint32_t DO_OFF = 4 * TILE;                   // 1 slot
   static constexpr uint32_t DS_OFF = 5 * TILE;                   // 128 x 128 16-bit, 2 chunks
   static constexpr uint32_t STG_OFF = DS_OFF + 2 * CHUNK;        // 4 warps x (32 rows x 128 B) fp32 staging
-  static constexpr uint32_t STAT_OFF = STG_OFF + 4 * 4096;       // 2 slots x (128 lse2 + 128 delta) fp32
+  static constexpr uint32_t STAT_OFF = STG_OFF + 4 * 4096;       // 2 slots x (128 -lse2 + 128 delta) fp32
   static constexpr uint32_t BAR_OFF = STAT_OFF + 2 * 1024;
   // kv_full q_full[2] q_empty[2] do_full do_empty s_full dp_full p_full ds_full
   // dq_full dq_empty dkv_full drain dq_done
@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict
     for (int w = G / 2; w > 0; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
     if (in && part == 0) {
       p.delta_w[row] = s < p.S ? acc : 0.f;
-      p.lse2_w[row] = s < p.S ? lse[(size_t)h * p.S + s] * 1.4426950408889634f : INFINITY;
+      p.nlse2_w[row] = s < p.S ? lse[(size_t)h * p.S + s] * -1.4426950408889634f : -INFINITY;
     }
   }
   // zero the dQ accumulator (16-byte stores) and the ordering counters
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(512, 1)
         for (int c = 0; c < C::CH; ++c)
           tma_load_3d(smem + C::Q_OFF + qs * C::TILE + c * C::CHUNK, &tm_q, &q_full[qs], c * 64, 128 * i, head);
         const size_t srow = (size_t)head * p.S_pad + 128 * i;
-        bulk_load(stats + qs * 256, p.lse2 + srow, 512, &q_full[qs]);
+        bulk_load(stats + qs * 256, p.nlse2 + srow, 512, &q_full[qs]);
         bulk_load(stats + qs * 256 + 128, p.delta + srow, 512, &q_full[qs]);
         ++q_issued;
         // dO_i into the dO slot
@@ -403,27 +403,33 @@ __global__ void __launch_bounds__(512, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const float* lse2 = stats + qs * 256;
-      const float* dlt = lse2 + 128;
+      const float* nl2 = stats + qs * 256;  // -LSE * log2(e) of the 128 queries
+      const float* dlt = nl2 + 128;         // D of the 128 queries
       // visible queries of this key row in tile i: q >= kv under the causal mask
       const int qlo = (CAUSAL && i == j) ? r : 0;
-      // ---- P phase (score columns 64*half .. +63)
-      uint32_t pk[32];
+      const bool masked = qlo > 64 * half || !kv_valid;  // some column of this half is invisible
+      // ---- P phase (score columns 64*half .. +63): P^T = 2^(S^T scale log2 e - LSE log2 e)
+      uint32_t sv[2][32];
+      tmem_ld32(tA + 64 * half, sv[0]);
+      tmem_ld32(tA + 64 * half + 32, sv[1]);
+      tmem_ld_wait(sv[0]);
+      tmem_ld_wait(sv[1]);
+      const uint64_t sl2x2 = f2(sl2, sl2);
+      uint32_t pk[32];  // P pairs rounded to 16 bits (the products' and dS's P)
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        const int c0 = 64 * half + 32 * ch;
-        uint32_t sv[32];
-        tmem_ld32(tA + c0, sv);
-        tmem_ld_wait(sv);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = c0 + 2 * e;
-          float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -lse2[c]));
-          float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -lse2[c + 1]));
+      for (int e = 0; e < 32; ++e) {
+        const int c = 64 * half + 2 * e;
+        const uint32_t* src = sv[e >> 4] + 2 * (e & 15);
+        const float2 nl = *reinterpret_cast<const float2*>(nl2 + c);
+        float p0, p1;
+        f2split(ffma2(f2(__uint_as_float(src[0]), __uint_as_float(src[1])), sl2x2, f2(nl.x, nl.y)), p0, p1);
+        p0 = ex2(p0);
+        p1 = ex2(p1);
+        if (masked) {
           if (c < qlo || !kv_valid) p0 = 0.f;
           if (c + 1 < qlo || !kv_valid) p1 = 0.f;
-          pk[16 * ch + e] = pack2<BF16>(p0, p1);
         }
+        pk[e] = pack2<BF16>(p0, p1);
       }
       // P^T pairs go to columns [64*half, 64*half + 32) of A (inside this
       // half's own score columns, already read)
@@ -431,24 +437,28 @@ __global__ void __launch_bounds__(512, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
-      // ---- dS phase
+      // ---- dS phase: dS^T = P^T (dP^T - D), P as rounded for the products
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, st & 1, BWD_SITE_DP));
       if (!ok) break;
       tc_fence_after();
+      uint32_t dv[2][32];
+      tmem_ld32(tB + 64 * half, dv[0]);
+      tmem_ld32(tB + 64 * half + 32, dv[1]);
+      tmem_ld_wait(dv[0]);
+      tmem_ld_wait(dv[1]);
       uint32_t dd[32];
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        const int c0 = 64 * half + 32 * ch;
-        uint32_t dv[32];
-        tmem_ld32(tB + c0, dv);
-        tmem_ld_wait(dv);
+      for (int e = 0; e < 32; ++e) {
+        const int c = 64 * half + 2 * e;
+        const uint32_t* src = dv[e >> 4] + 2 * (e & 15);
+        const float2 dl = *reinterpret_cast<const float2*>(dlt + c);
+        const uint64_t dpd = fadd2(f2(__uint_as_float(src[0]), __uint_as_float(src[1])), f2(-dl.x, -dl.y));
+        float a, b;
+        f2split(fmul2(widen2<BF16>(pk[e]), dpd), a, b);
+        dd[e] = pack2<BF16>(a, b);
+      }
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = c0 + 2 * e;
-          const float2 pp = unpack2<BF16>(pk[16 * ch + e]);
-          dd[16 * ch + e] = pack2<BF16>(pp.x * (__uint_as_float(dv[2 * e]) - dlt[c]),
-                                        pp.y * (__uint_as_float(dv[2 * e + 1]) - dlt[c + 1]));
-        }
+      for (int ch = 0; ch < 2; ++ch) {
         // dS row r (key), 32 query columns: MN-major A operand of dQ = dS K,
         // [key][query] with queries contiguous, 64-query chunk = half, 128-B swizzled
         const uint32_t base = half * C::CHUNK + r * 128 + ch * 64;
