@@ -27,7 +27,8 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = ran
 FA_BF16, FA_FP16 = 0, 1
 
 EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
-           "fa_bwd_finish", "fa_bwd_noalloc", "fa_status_string", "fa_check_device_error", "fa_launch_count")
+           "fa_bwd_finish", "fa_bwd_noalloc", "fa_bwd_varlen_workspace_size", "fa_bwd_varlen", "fa_status_string",
+           "fa_check_device_error", "fa_launch_count")
 
 # Fixed scratch size of fa_bwd_noalloc (FA_BWD_NOALLOC_SCRATCH_BYTES in include/fa.h).
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -68,6 +69,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_bwd_finish.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
     lib.fa_bwd_noalloc.restype = i
+    lib.fa_bwd_varlen_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa_bwd_varlen_workspace_size.restype = sz
+    lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp, sz, vp]
+    lib.fa_bwd_varlen.restype = i
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_check_device_error.argtypes = [vp]
@@ -117,6 +122,17 @@ def fa_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, causal, d
                    stream) -> int:
     return load_library().fa_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, int(causal), dt,
                                          int(deterministic), stream)
+
+
+def fa_bwd_varlen_workspace_size(nseq, max_seqlen, total, H, D) -> int:
+    return load_library().fa_bwd_varlen_workspace_size(nseq, max_seqlen, total, H, D)
+
+
+def fa_bwd_varlen(q, k, v, o, dO, lse, dq, dk, dv, cu_seqlens, nseq, max_seqlen, total, H, D, scale, causal, dt,
+                  deterministic, workspace, workspace_bytes, stream) -> int:
+    return load_library().fa_bwd_varlen(q, k, v, o, dO, lse, dq, dk, dv, cu_seqlens, nseq, max_seqlen, total, H, D,
+                                        scale, int(causal), dt, int(deterministic), workspace, workspace_bytes,
+                                        stream)
 
 
 def fa_status_string(status: int) -> str:
@@ -211,6 +227,29 @@ def backward(q, k, v, o, do, lse, causal: bool, scale: float | None = None, dete
                 workspace.data_ptr(), workspace.numel(), _stream(stream))
     if st != FA_OK:
         raise FAError(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def backward_varlen(q, k, v, o, do, lse, cu_seqlens, max_seqlen: int, causal: bool, scale: float | None = None,
+                    deterministic: bool = False, workspace=None, stream=None):
+    """dQ, dK, dV of a packed [H, T, D] batch given fa_fwd_varlen's O and LSE."""
+    import torch
+    H, T, D = q.shape
+    _check((q, k, v, o, do), q.shape)
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
+        raise TypeError("cu_seqlens must be a CUDA int32 tensor")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    nseq = cu_seqlens.numel() - 1
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nbytes = fa_bwd_varlen_workspace_size(nseq, int(max_seqlen), T, H, D)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(max(nbytes, 1), device=q.device, dtype=torch.uint8)
+    st = fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu_seqlens.data_ptr(), nseq, int(max_seqlen), T,
+                       H, D, scale, causal, _dt(q), deterministic, workspace.data_ptr(), workspace.numel(),
+                       _stream(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd_varlen")
     return dq, dk, dv
 
 

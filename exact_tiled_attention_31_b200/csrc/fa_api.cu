@@ -150,19 +150,22 @@ struct WsLayout {
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
-WsLayout ws_layout(long long heads, long long S, int D) {
+// heads x rows token rows in memory; statistics padded per sequence to
+// ceil(S / 128) * 128 rows (S = the longest sequence)
+WsLayout ws_layout(long long heads, long long nseq, long long S, long long rows, int D) {
   const long long n_q = (S + 127) / 128, S_pad = n_q * 128;
   WsLayout w;
   w.dq_acc = 0;
-  w.lse2 = up256((size_t)heads * S * D * 4);
-  w.delta = w.lse2 + up256((size_t)heads * S_pad * 4);
-  w.sem = w.delta + up256((size_t)heads * S_pad * 4);
-  w.total = w.sem + up256((size_t)heads * n_q * 4);
+  w.lse2 = up256((size_t)heads * rows * D * 4);
+  w.delta = w.lse2 + up256((size_t)heads * nseq * S_pad * 4);
+  w.sem = w.delta + up256((size_t)heads * nseq * S_pad * 4);
+  w.total = w.sem + up256((size_t)heads * nseq * n_q * 4);
   return w;
 }
 
-fa::BwdParams bwd_params(int heads, int S, int D, float scale, int deterministic, uint8_t* ws, void* dk, void* dv) {
-  const WsLayout w = ws_layout(heads, S, D);
+fa::BwdParams bwd_params(int heads, int nseq, int S, int rows, const int* cu, int D, float scale, int deterministic,
+                         uint8_t* ws, void* dk, void* dv) {
+  const WsLayout w = ws_layout(heads, nseq, S, rows, D);
   fa::BwdParams p;
   p.dk = dk;
   p.dv = dv;
@@ -170,8 +173,11 @@ fa::BwdParams bwd_params(int heads, int S, int D, float scale, int deterministic
   p.nlse2 = p.nlse2_w = reinterpret_cast<float*>(ws + w.lse2);
   p.delta = p.delta_w = reinterpret_cast<float*>(ws + w.delta);
   p.sem = reinterpret_cast<uint32_t*>(ws + w.sem);
+  p.cu_seqlens = cu;
   p.heads = heads;
   p.S = S;
+  p.rows = rows;
+  p.nseq = nseq;
   p.n_q = (S + 127) / 128;
   p.S_pad = p.n_q * 128;
   p.scale = scale;
@@ -181,41 +187,71 @@ fa::BwdParams bwd_params(int heads, int S, int D, float scale, int deterministic
 }
 
 template <int D, bool BF16>
-fa_status launch_bwd_pre(const void* o, const void* dO, const float* lse, const fa::BwdParams& p, cudaStream_t st) {
-  fa::bwd_pre_kernel<D, BF16><<<sm_count() * 8, 256, 0, st>>>(static_cast<const uint16_t*>(o),
-                                                                static_cast<const uint16_t*>(dO), lse, p);
+fa_status launch_bwd_pre(const void* o, const void* dO, const float* lse, const fa::BwdParams& p, bool varlen,
+                         cudaStream_t st) {
+  const uint16_t* o16 = static_cast<const uint16_t*>(o);
+  const uint16_t* do16 = static_cast<const uint16_t*>(dO);
+  if (varlen)
+    fa::bwd_pre_kernel<D, BF16, true><<<sm_count() * 8, 256, 0, st>>>(o16, do16, lse, p);
+  else
+    fa::bwd_pre_kernel<D, BF16, false><<<sm_count() * 8, 256, 0, st>>>(o16, do16, lse, p);
+  g_launches.fetch_add(1);
+  return from_cuda(cudaGetLastError());
+}
+
+template <int D, bool BF16, bool CAUSAL, bool VARLEN>
+fa_status launch_bwd_main_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const CUtensorMap& mdo, const CUtensorMap& mdq, const fa::BwdParams& p, cudaStream_t st) {
+  using C = fa::BwdCfg<D>;
+  const long long grid = (long long)p.n_q * p.nseq * p.heads;
+  if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  if (set_smem<fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN>>(C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
+  fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN><<<(unsigned)grid, 512, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, p);
   g_launches.fetch_add(1);
   return from_cuda(cudaGetLastError());
 }
 
 template <int D, bool BF16>
 fa_status launch_bwd_main(const void* q, const void* k, const void* v, const void* dO, const fa::BwdParams& p,
-                          bool causal, cudaStream_t st) {
-  using C = fa::BwdCfg<D>;
+                          bool causal, bool varlen, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mdo, mdq;
-  if (!make_map(&mq, q, D, p.S, p.heads, BF16) || !make_map(&mk, k, D, p.S, p.heads, BF16) ||
-      !make_map(&mv, v, D, p.S, p.heads, BF16) || !make_map(&mdo, dO, D, p.S, p.heads, BF16) ||
-      !make_map_f32(&mdq, p.dq_acc, D, p.S, p.heads))
+  if (!make_map(&mq, q, D, p.rows, p.heads, BF16) || !make_map(&mk, k, D, p.rows, p.heads, BF16) ||
+      !make_map(&mv, v, D, p.rows, p.heads, BF16) || !make_map(&mdo, dO, D, p.rows, p.heads, BF16) ||
+      !make_map_f32(&mdq, p.dq_acc, D, p.rows, p.heads))
     return FA_ERR_CUDA;
-  const long long grid = (long long)p.n_q * p.heads;
-  if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-  cudaError_t e = causal ? set_smem<fa::bwd_main_kernel<D, BF16, true>>(C::SMEM)
-                         : set_smem<fa::bwd_main_kernel<D, BF16, false>>(C::SMEM);
-  if (e != cudaSuccess) return FA_ERR_CUDA;
-  if (causal)
-    fa::bwd_main_kernel<D, BF16, true><<<(unsigned)grid, 512, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, p);
-  else
-    fa::bwd_main_kernel<D, BF16, false><<<(unsigned)grid, 512, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, p);
-  g_launches.fetch_add(1);
-  return from_cuda(cudaGetLastError());
+  if (varlen)
+    return causal ? launch_bwd_main_t<D, BF16, true, true>(mq, mk, mv, mdo, mdq, p, st)
+                  : launch_bwd_main_t<D, BF16, false, true>(mq, mk, mv, mdo, mdq, p, st);
+  return causal ? launch_bwd_main_t<D, BF16, true, false>(mq, mk, mv, mdo, mdq, p, st)
+                : launch_bwd_main_t<D, BF16, false, false>(mq, mk, mv, mdo, mdq, p, st);
 }
 
 template <bool BF16>
 fa_status launch_bwd_post(void* dq, const fa::BwdParams& p, int D, cudaStream_t st) {
-  const long long n8 = (long long)p.heads * p.S * D / 8;
+  const long long n8 = (long long)p.heads * p.rows * D / 8;
   fa::bwd_post_kernel<BF16><<<sm_count() * 8, 256, 0, st>>>(p.dq_acc, static_cast<uint16_t*>(dq), n8, p.scale);
   g_launches.fetch_add(1);
   return from_cuda(cudaGetLastError());
+}
+
+// The three backward launches over prepared parameters (dense or packed).
+fa_status run_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                  void* dq, const fa::BwdParams& p, int D, bool causal, bool bf16, bool varlen, cudaStream_t st) {
+  fa_status c;
+  if (D == 64)
+    c = bf16 ? launch_bwd_pre<64, true>(o, dO, lse, p, varlen, st) : launch_bwd_pre<64, false>(o, dO, lse, p, varlen, st);
+  else
+    c = bf16 ? launch_bwd_pre<128, true>(o, dO, lse, p, varlen, st)
+             : launch_bwd_pre<128, false>(o, dO, lse, p, varlen, st);
+  if (c != FA_OK) return c;
+  if (D == 64)
+    c = bf16 ? launch_bwd_main<64, true>(q, k, v, dO, p, causal, varlen, st)
+             : launch_bwd_main<64, false>(q, k, v, dO, p, causal, varlen, st);
+  else
+    c = bf16 ? launch_bwd_main<128, true>(q, k, v, dO, p, causal, varlen, st)
+             : launch_bwd_main<128, false>(q, k, v, dO, p, causal, varlen, st);
+  if (c != FA_OK) return c;
+  return bf16 ? launch_bwd_post<true>(dq, p, D, st) : launch_bwd_post<false>(dq, p, D, st);
 }
 
 // shared checks of the backward entry points: sizes, dtype, workspace
@@ -226,7 +262,7 @@ fa_status bwd_common_checks(int B, int H, int S, int D, fa_dtype dt, const void*
   if ((long long)B * H > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   if (B == 0 || H == 0 || S == 0) return FA_OK;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_INVALID_ARG;
-  size_t need = ws_layout((long long)B * H, S, D).total;
+  size_t need = ws_layout((long long)B * H, 1, S, S, D).total;
   if (workspace_bytes < need) return FA_ERR_INVALID_ARG;
   return FA_OK;
 }
@@ -298,7 +334,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
 
 size_t fa_bwd_workspace_size(int B, int H, int S, int D) {
   if (B <= 0 || H <= 0 || S <= 0 || (D != 64 && D != 128)) return 0;
-  return ws_layout((long long)B * H, S, D).total;
+  return ws_layout((long long)B * H, 1, S, S, D).total;
 }
 
 fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int S, int D,
@@ -306,10 +342,14 @@ fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int
   fa_status c = bwd_common_checks(B, H, S, D, dt, workspace, workspace_bytes);
   if (c != FA_OK || B == 0 || H == 0 || S == 0) return c;
   if (!ptrs_ok({o, dO, lse})) return FA_ERR_INVALID_ARG;
-  const fa::BwdParams p = bwd_params(B * H, S, D, 1.f, 0, static_cast<uint8_t*>(workspace), nullptr, nullptr);
+  const fa::BwdParams p =
+      bwd_params(B * H, 1, S, S, nullptr, D, 1.f, 0, static_cast<uint8_t*>(workspace), nullptr, nullptr);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 64) return dt == FA_BF16 ? launch_bwd_pre<64, true>(o, dO, lse, p, st) : launch_bwd_pre<64, false>(o, dO, lse, p, st);
-  return dt == FA_BF16 ? launch_bwd_pre<128, true>(o, dO, lse, p, st) : launch_bwd_pre<128, false>(o, dO, lse, p, st);
+  if (D == 64)
+    return dt == FA_BF16 ? launch_bwd_pre<64, true>(o, dO, lse, p, false, st)
+                         : launch_bwd_pre<64, false>(o, dO, lse, p, false, st);
+  return dt == FA_BF16 ? launch_bwd_pre<128, true>(o, dO, lse, p, false, st)
+                       : launch_bwd_pre<128, false>(o, dO, lse, p, false, st);
 }
 
 fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B, int H,
@@ -320,13 +360,15 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* d
   if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
   if (B == 0 || H == 0 || S == 0) return FA_OK;
   if (!ptrs_ok({q, k, v, dO, dk, dv})) return FA_ERR_INVALID_ARG;
-  const fa::BwdParams p =
-      bwd_params(B * H, S, D, scale, deterministic != 0, static_cast<uint8_t*>(workspace), dk, dv);
+  const fa::BwdParams p = bwd_params(B * H, 1, S, S, nullptr, D, scale, deterministic != 0,
+                                     static_cast<uint8_t*>(workspace), dk, dv);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool cz = causal != 0;
   if (D == 64)
-    return dt == FA_BF16 ? launch_bwd_main<64, true>(q, k, v, dO, p, cz, st) : launch_bwd_main<64, false>(q, k, v, dO, p, cz, st);
-  return dt == FA_BF16 ? launch_bwd_main<128, true>(q, k, v, dO, p, cz, st) : launch_bwd_main<128, false>(q, k, v, dO, p, cz, st);
+    return dt == FA_BF16 ? launch_bwd_main<64, true>(q, k, v, dO, p, cz, false, st)
+                         : launch_bwd_main<64, false>(q, k, v, dO, p, cz, false, st);
+  return dt == FA_BF16 ? launch_bwd_main<128, true>(q, k, v, dO, p, cz, false, st)
+                       : launch_bwd_main<128, false>(q, k, v, dO, p, cz, false, st);
 }
 
 fa_status fa_bwd_finish(void* dq, int B, int H, int S, int D, float scale, fa_dtype dt, void* workspace,
@@ -336,7 +378,8 @@ fa_status fa_bwd_finish(void* dq, int B, int H, int S, int D, float scale, fa_dt
   if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
   if (B == 0 || H == 0 || S == 0) return FA_OK;
   if (!ptrs_ok({dq})) return FA_ERR_INVALID_ARG;
-  const fa::BwdParams p = bwd_params(B * H, S, D, scale, 0, static_cast<uint8_t*>(workspace), nullptr, nullptr);
+  const fa::BwdParams p =
+      bwd_params(B * H, 1, S, S, nullptr, D, scale, 0, static_cast<uint8_t*>(workspace), nullptr, nullptr);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return dt == FA_BF16 ? launch_bwd_post<true>(dq, p, D, st) : launch_bwd_post<false>(dq, p, D, st);
 }
@@ -373,6 +416,30 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   if (!scratch) return FA_ERR_CUDA;
   return fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, causal, dt, deterministic, scratch,
                 (size_t)FA_BWD_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+size_t fa_bwd_varlen_workspace_size(int nseq, int max_seqlen, int total, int H, int D) {
+  if (nseq <= 0 || max_seqlen <= 0 || total <= 0 || H <= 0 || (D != 64 && D != 128)) return 0;
+  return ws_layout(H, nseq, max_seqlen, total, D).total;
+}
+
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                        const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens, int nseq,
+                        int max_seqlen, int total, int H, int D, float scale, int causal, fa_dtype dt,
+                        int deterministic, void* workspace, size_t workspace_bytes, void* stream) {
+  if (nseq < 0 || max_seqlen < 0 || total < 0 || H < 0) return FA_ERR_INVALID_ARG;
+  if (dt != FA_BF16 && dt != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (nseq == 0 || H == 0 || total == 0 || max_seqlen == 0) return FA_OK;
+  if (max_seqlen > total) return FA_ERR_INVALID_ARG;
+  if (!ptrs_ok({q, k, v, o, dO, lse, dq, dk, dv}) || !cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < ws_layout(H, nseq, max_seqlen, total, D).total) return FA_ERR_INVALID_ARG;
+  const fa::BwdParams p = bwd_params(H, nseq, max_seqlen, total, cu_seqlens, D, scale, deterministic != 0,
+                                     static_cast<uint8_t*>(workspace), dk, dv);
+  return run_bwd(q, k, v, o, dO, lse, dq, p, D, causal != 0, dt == FA_BF16, true, static_cast<cudaStream_t>(stream));
 }
 
 const char* fa_status_string(fa_status s) {

@@ -15,7 +15,8 @@
 //   bwd_pre   D_i = dO_i . O_i (fp32, warp-shuffle reduction), -LSE_i*log2(e)
 //             into a 128-row-padded copy, zero the fp32 dQ accumulator and
 //             the ordering counters.
-//   bwd_main  one CTA per 128-row key/value tile j of one head (512 threads):
+//   bwd_main  one CTA per 128-row key/value tile j of one head (and, for a
+//             packed batch, one sequence; 512 threads):
 //               warp 0     TMA producer: K_j, V_j once; then Q_i (+ the padded
 //                          LSE/D rows of tile i) into a 2-slot ring and dO_i
 //                          into its own slot.
@@ -45,7 +46,11 @@
 //                          tile i one at a time in increasing j.
 //   bwd_post  dQ = scale * accumulator, rounded to the input dtype.
 // Causal: key tile j only meets query tiles i >= j; only the diagonal tile
-// is masked element-wise.
+// is masked element-wise.  Packed batches ([H, T, D], cu_seqlens): every
+// sequence is its own problem with tiles counted from its first token; keys
+// past its end get P = 0 and query rows past its end carry LSE padding of
+// -inf, so their dS rows are exactly 0 and nothing leaks into the next
+// sequence's rows (the fp32 reductions of those zero rows add 0).
 #pragma once
 
 #include "sm100.cuh"
@@ -53,15 +58,20 @@
 namespace fa {
 
 struct BwdParams {
-  void* dk;                // [heads, S, D]
-  void* dv;                // [heads, S, D]
-  float* dq_acc;           // [heads, S, D] fp32
-  const float* nlse2;      // [heads, S_pad]  -LSE * log2(e), -inf in padding rows
-  const float* delta;      // [heads, S_pad]  D_i, 0 in padding rows
+  void* dk;                // [heads, rows, D]
+  void* dv;                // [heads, rows, D]
+  float* dq_acc;           // [heads, rows, D] fp32
+  const float* nlse2;      // [heads, nseq, S_pad]  -LSE * log2(e), -inf in padding rows
+  const float* delta;      // [heads, nseq, S_pad]  D_i, 0 in padding rows
   float* nlse2_w;          // the same two buffers, written by bwd_pre
   float* delta_w;
-  uint32_t* sem;           // [heads, n_q] ordering counters (deterministic mode)
-  int heads, S, S_pad, n_q;
+  uint32_t* sem;           // [heads, nseq, n_q] ordering counters (deterministic mode)
+  const int* cu_seqlens;   // packed batch only: device int32 [nseq + 1]
+  int heads;               // dense: B*H, packed: H
+  int S;                   // dense: S, packed: max_seqlen
+  int rows;                // rows of one head slice in memory: S or total
+  int nseq;                // dense: 1
+  int S_pad, n_q;          // ceil(S / 128) * 128, ceil(S / 128)
   float scale, scale_log2;
   int deterministic;
 };
@@ -95,23 +105,32 @@ enum : uint32_t {
 // ---------------------------------------------------------------------------
 // bwd_pre: one group of D/8 lanes per row, 16-byte loads, shuffle reduction.
 // ---------------------------------------------------------------------------
-template <int D, bool BF16>
+template <int D, bool BF16, bool VARLEN>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dO,
                                                       const float* __restrict__ lse, BwdParams p) {
   constexpr int G = D / 8;  // lanes per row
-  const long long work = (long long)p.heads * p.S_pad * G;
+  const long long work = (long long)p.heads * p.nseq * p.S_pad * G;
   const long long bound = (work + 31) / 32 * 32;  // whole warps take the same trips
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long nthreads = (long long)gridDim.x * blockDim.x;
   for (long long idx = gtid; idx < bound; idx += nthreads) {
     const bool in = idx < work;
-    const long long row = idx / G;
+    const long long row = idx / G;  // padded row: (head * nseq + seq) * S_pad + s
     const int part = (int)(idx % G);
-    const int h = in ? (int)(row / p.S_pad) : 0;
-    const int s = in ? (int)(row % p.S_pad) : p.S;
+    const long long hs = in ? row / p.S_pad : 0;
+    const int h = (int)(hs / p.nseq);
+    const int seq = (int)(hs - (long long)h * p.nseq);
+    int base = 0, len = p.S;
+    if constexpr (VARLEN) {
+      base = p.cu_seqlens[seq];
+      len = p.cu_seqlens[seq + 1] - base;
+    }
+    const int s = in ? (int)(row - hs * p.S_pad) : len;
+    const bool valid = s < len;
+    const size_t tok = (size_t)h * p.rows + base + s;  // token row in memory (valid rows only)
     float acc = 0.f;
-    if (s < p.S) {
-      const size_t off = ((size_t)h * p.S + s) * D + part * 8;
+    if (valid) {
+      const size_t off = tok * D + part * 8;
       const uint4 a = *reinterpret_cast<const uint4*>(o + off);
       const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
       const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
@@ -126,15 +145,15 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict
 #pragma unroll
     for (int w = G / 2; w > 0; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
     if (in && part == 0) {
-      p.delta_w[row] = s < p.S ? acc : 0.f;
-      p.nlse2_w[row] = s < p.S ? lse[(size_t)h * p.S + s] * -1.4426950408889634f : -INFINITY;
+      p.delta_w[row] = valid ? acc : 0.f;
+      p.nlse2_w[row] = valid ? lse[tok] * -1.4426950408889634f : -INFINITY;
     }
   }
   // zero the dQ accumulator (16-byte stores) and the ordering counters
-  const long long n4 = (long long)p.heads * p.S * D / 4;
+  const long long n4 = (long long)p.heads * p.rows * D / 4;
   float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
   for (long long i = gtid; i < n4; i += nthreads) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  const long long ns = (long long)p.heads * p.n_q;
+  const long long ns = (long long)p.heads * p.nseq * p.n_q;
   for (long long i = gtid; i < ns; i += nthreads) p.sem[i] = 0u;
 }
 
@@ -190,17 +209,29 @@ __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
 // ---------------------------------------------------------------------------
 // bwd_main
 // ---------------------------------------------------------------------------
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<D>;
-  const int j = blockIdx.x / p.heads;  // key/value tile (ascending: longest causal work first)
-  const int head = blockIdx.x - j * p.heads;
+  // work unit: (key/value tile j, sequence, head), ascending j = longest causal work first
+  const int per_j = p.nseq * p.heads;
+  const int j = blockIdx.x / per_j;
+  const int rem = blockIdx.x - j * per_j;
+  const int seq = rem / p.heads;
+  const int head = rem - seq * p.heads;
+  int row_base = 0, seq_len = p.S;  // first token row and length of this sequence
+  if constexpr (VARLEN) {
+    row_base = p.cu_seqlens[seq];
+    seq_len = p.cu_seqlens[seq + 1] - row_base;
+  }
+  if (128 * j >= seq_len) return;  // uniform over the CTA, before any set-up
+  const int n_q = (seq_len + 127) / 128;
   const int i_begin = CAUSAL ? j : 0;
-  const int n_steps = p.n_q - i_begin;
-  const int kv_row0 = 128 * j;
+  const int n_steps = n_q - i_begin;
+  const int kv_row0 = 128 * j;  // inside the sequence
+  const size_t stat_row0 = ((size_t)head * p.nseq + seq) * p.S_pad;  // padded statistics of this sequence
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -254,7 +285,7 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem = *tmem_holder;
 
   // register split over 512 threads launched with 128 each (65536):
-  // 128 x 56 (warps 0-3) + 256 x 152 (P/dS) + 128 x 144 (dQ) = 64512.
+  // 128 x 56 (warps 0-3) + 256 x 136 (P/dS) + 128 x 176 (dQ) = 64512.
   // Each warpgroup changes its budget inside its own branch.
   if (warp < 4) {
   regs_dec<56>();
@@ -267,8 +298,8 @@ __global__ void __launch_bounds__(512, 1)
       tma_prefetch_desc(&tm_do);
       mbar_expect_tx(kv_full, 2 * C::TILE);
       for (int c = 0; c < C::CH; ++c) {
-        tma_load_3d(smem + C::K_OFF + c * C::CHUNK, &tm_k, kv_full, c * 64, kv_row0, head);
-        tma_load_3d(smem + C::V_OFF + c * C::CHUNK, &tm_v, kv_full, c * 64, kv_row0, head);
+        tma_load_3d(smem + C::K_OFF + c * C::CHUNK, &tm_k, kv_full, c * 64, row_base + kv_row0, head);
+        tma_load_3d(smem + C::V_OFF + c * C::CHUNK, &tm_v, kv_full, c * 64, row_base + kv_row0, head);
       }
       bool ok = true;
       int q_issued = 0, do_issued = 0;
@@ -279,8 +310,9 @@ __global__ void __launch_bounds__(512, 1)
         if (st >= 2 && !(ok = mbar_wait(&q_empty[qs], ((st >> 1) - 1) & 1, BWD_SITE_PROD))) break;
         mbar_expect_tx(&q_full[qs], C::TILE + 1024u);
         for (int c = 0; c < C::CH; ++c)
-          tma_load_3d(smem + C::Q_OFF + qs * C::TILE + c * C::CHUNK, &tm_q, &q_full[qs], c * 64, 128 * i, head);
-        const size_t srow = (size_t)head * p.S_pad + 128 * i;
+          tma_load_3d(smem + C::Q_OFF + qs * C::TILE + c * C::CHUNK, &tm_q, &q_full[qs], c * 64,
+                      row_base + 128 * i, head);
+        const size_t srow = stat_row0 + 128 * i;
         bulk_load(stats + qs * 256, p.nlse2 + srow, 512, &q_full[qs]);
         bulk_load(stats + qs * 256 + 128, p.delta + srow, 512, &q_full[qs]);
         ++q_issued;
@@ -288,7 +320,7 @@ __global__ void __launch_bounds__(512, 1)
         if (st >= 1 && !(ok = mbar_wait(do_empty, (st - 1) & 1, BWD_SITE_PROD))) break;
         mbar_expect_tx(do_full, C::TILE);
         for (int c = 0; c < C::CH; ++c)
-          tma_load_3d(smem + C::DO_OFF + c * C::CHUNK, &tm_do, do_full, c * 64, 128 * i, head);
+          tma_load_3d(smem + C::DO_OFF + c * C::CHUNK, &tm_do, do_full, c * 64, row_base + 128 * i, head);
         ++do_issued;
       }
       // no tile copy may still be landing in shared memory at exit
@@ -382,7 +414,7 @@ __global__ void __launch_bounds__(512, 1)
     __syncwarp();
   }
   } else if (warp < 12) {
-    regs_inc<152>();
+    regs_inc<136>();
     // ------------------------------------------------------------ P / dS
     // One thread per key row and half of the 128 query columns: warps 4-7
     // take queries 0-63, warps 8-11 queries 64-127.  P and dS are
@@ -392,7 +424,7 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tA = tmem + lane_off + C::TM_A, tB = tmem + lane_off + C::TM_B;
     const int kv = kv_row0 + r;
-    const bool kv_valid = kv < p.S;
+    const bool kv_valid = kv < seq_len;
     const float sl2 = p.scale_log2;
     uint8_t* ds_smem = smem + C::DS_OFF;
     bool ok = true;
@@ -479,7 +511,7 @@ __global__ void __launch_bounds__(512, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dkv_full, 0, BWD_SITE_DKV));
     if (ok) {
       tc_fence_after();
-      const size_t grow = ((size_t)head * p.S + kv) * D;
+      const size_t grow = ((size_t)head * p.rows + row_base + kv) * D;
       {
         const int which = half;  // half 0 writes dV, half 1 writes scale * dK
         uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(which ? p.dk : p.dv) + grow);
@@ -503,7 +535,7 @@ __global__ void __launch_bounds__(512, 1)
       }
     }
   } else {
-    regs_inc<144>();
+    regs_inc<176>();
     // ------------------------------------------------------------ dQ (one thread per query row)
     const int c = threadIdx.x - 384;                 // query row within the tile = TMEM lane
     const int wq = warp - 12;                        // this warp's 32 rows: 32*wq ..
@@ -534,13 +566,13 @@ __global__ void __launch_bounds__(512, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_reduce_add_3d(&tm_dq, stg, 32 * cc, 128 * i + 32 * wq, head);
+            tma_reduce_add_3d(&tm_dq, stg, 32 * cc, row_base + 128 * i + 32 * wq, head);
             bulk_commit();
           }
         }
       } else {
         // key tiles add into query tile i in increasing j: wait for our turn
-        uint32_t* sem = p.sem + (size_t)head * p.n_q + i;
+        uint32_t* sem = p.sem + ((size_t)head * p.nseq + seq) * p.n_q + i;
         bool ok = true;
         if (ld_acquire_gpu(sem) != (uint32_t)j) {
           const uint64_t t0 = global_ns();
@@ -552,8 +584,8 @@ __global__ void __launch_bounds__(512, 1)
             }
           }
         }
-        if (ok && q < p.S) {
-          float4* dst = reinterpret_cast<float4*>(p.dq_acc + ((size_t)head * p.S + q) * D);
+        if (ok && q < seq_len) {  // rows of this sequence only
+          float4* dst = reinterpret_cast<float4*>(p.dq_acc + ((size_t)head * p.rows + row_base + q) * D);
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc)
 #pragma unroll

@@ -120,6 +120,29 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int deterministic, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward pass over a packed batch of variable-length sequences (the
+ * gradients of fa_fwd_varlen's output; same formulas as fa_bwd, each
+ * sequence on its own, causal counted from its first token).
+ *   q, k, v, o, dO : [H, total, D];  lse : fp32 [H, total] from fa_fwd_varlen.
+ *   dq, dk, dv     : [H, total, D] outputs, same dtype.
+ *   cu_seqlens, nseq, max_seqlen, total : as for fa_fwd_varlen.
+ *   workspace : caller-owned device buffer of at least
+ *               fa_bwd_varlen_workspace_size(nseq, max_seqlen, total, H, D)
+ *               bytes, 256-byte aligned; contents on entry do not matter.
+ *   deterministic : as for fa_bwd (key tiles of one sequence add into a query
+ *               tile in increasing order).
+ * Cites: "Flash Attention 的算法设计原理", "练习口述回答" (variable-length inputs
+ * are a branch to test on their own) and "核心机制" (recompute P from the
+ * saved statistics).  nseq, H, total or max_seqlen equal to 0 is a no-op.
+ */
+size_t fa_bwd_varlen_workspace_size(int nseq, int max_seqlen, int total, int H, int D);
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                        const float* lse, void* dq, void* dk, void* dv,
+                        const int* cu_seqlens, int nseq, int max_seqlen, int total,
+                        int H, int D, float scale, int causal, fa_dtype dt,
+                        int deterministic, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The three launches fa_bwd makes, exposed for callers that want to place
  * or time them separately (same arguments, same rules, same workspace; they
  * must run in this order on one stream):

@@ -94,3 +94,30 @@ def test_missing_library_fails_loudly(tmp_path):
             fa.api.load_library(str(tmp_path / "nope.so"))
     finally:
         fa.api._lib = saved
+
+
+def test_bwd_varlen_workspace_and_argument_errors(lib):
+    def up(x):
+        return (x + 255) // 256 * 256
+    nseq, mx, T, H, D = 3, 300, 500, 4, 128
+    spad = (mx + 127) // 128 * 128
+    expect = up(H * T * D * 4) + 2 * up(H * nseq * spad * 4) + up(H * nseq * (spad // 128) * 4)
+    assert fa.fa_bwd_varlen_workspace_size(nseq, mx, T, H, D) == expect
+    assert fa.fa_bwd_varlen_workspace_size(nseq, mx, T, H, 96) == 0
+    assert fa.fa_bwd_varlen_workspace_size(0, mx, T, H, D) == 0
+    A = 1 << 20
+    ws = fa.fa_bwd_varlen_workspace_size(2, 50, 100, 1, 64)
+
+    def call(**kw):
+        a = dict(cu=A, nseq=2, mx=50, T=100, H=1, D=64, scale=0.1, causal=1, dt=0, det=0, ws=A, wsb=ws, dq=A)
+        a.update(kw)
+        return fa.fa_bwd_varlen(A, A, A, A, A, A, a["dq"], A, A, a["cu"], a["nseq"], a["mx"], a["T"], a["H"], a["D"],
+                                a["scale"], a["causal"], a["dt"], a["det"], a["ws"], a["wsb"], None)
+    assert call(mx=300) == fa.api.FA_ERR_INVALID_ARG         # longest sequence beyond the pack
+    assert call(cu=A + 2) == fa.api.FA_ERR_INVALID_ARG       # misaligned offsets
+    assert call(dq=A + 8) == fa.api.FA_ERR_INVALID_ARG       # misaligned output
+    assert call(ws=A + 64) == fa.api.FA_ERR_INVALID_ARG      # workspace not 256-byte aligned
+    assert call(wsb=ws - 1) == fa.api.FA_ERR_INVALID_ARG     # workspace too small
+    assert call(D=80) == fa.api.FA_ERR_UNSUPPORTED
+    assert call(scale=-1.0) == fa.api.FA_ERR_INVALID_ARG
+    assert call(nseq=0) == fa.api.FA_OK                       # empty pack: nothing to do
