@@ -203,7 +203,10 @@ template <int D, bool BF16, bool CAUSAL, bool VARLEN>
 fa_status launch_bwd_main_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const CUtensorMap& mdo, const CUtensorMap& mdq, const fa::BwdParams& p, cudaStream_t st) {
   using C = fa::BwdCfg<D>;
-  const long long grid = (long long)p.n_q * p.nseq * p.heads;
+  // groups of kBwdGroup (sequence, head) slices, n_q key tiles each
+  const long long units = (long long)p.nseq * p.heads;
+  const long long groups = (units + fa::kBwdGroup - 1) / fa::kBwdGroup;
+  const long long grid = groups * fa::kBwdGroup * p.n_q;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   if (set_smem<fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN>>(C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
   fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN><<<(unsigned)grid, 512, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, p);

@@ -96,6 +96,9 @@ struct BwdCfg {
   static constexpr uint32_t TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
 };
 
+// (sequence, head) slices per group of the backward's block order
+constexpr int kBwdGroup = 4;
+
 enum : uint32_t {
   BWD_SITE_PROD = 0x200, BWD_SITE_KV = 0x201, BWD_SITE_Q = 0x202, BWD_SITE_DO = 0x203, BWD_SITE_P = 0x204,
   BWD_SITE_DS = 0x205, BWD_SITE_DQE = 0x206, BWD_SITE_S = 0x207, BWD_SITE_DP = 0x208, BWD_SITE_DQF = 0x209,
@@ -215,12 +218,20 @@ __global__ void __launch_bounds__(512, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<D>;
-  // work unit: (key/value tile j, sequence, head), ascending j = longest causal work first
-  const int per_j = p.nseq * p.heads;
-  const int j = blockIdx.x / per_j;
-  const int rem = blockIdx.x - j * per_j;
-  const int seq = rem / p.heads;
-  const int head = rem - seq * p.heads;
+  // work unit: (key/value tile j, sequence, head).  Blocks walk groups of
+  // kBwdGroup (sequence, head) slices; inside a group, ascending j (longest
+  // causal work first).  Only a few slices are live at a time, so their fp32
+  // dQ accumulators and Q/K/V/dO tiles stay in L2, where the dQ reductions
+  // run about twice as fast as against device memory.
+  const int units = p.nseq * p.heads;
+  const int group = blockIdx.x / (kBwdGroup * p.n_q);
+  const int rg = blockIdx.x - group * (kBwdGroup * p.n_q);
+  const int gsize = min(kBwdGroup, units - group * kBwdGroup);
+  const int j = rg / gsize;
+  if (j >= p.n_q) return;  // the last group may be smaller than kBwdGroup
+  const int unit = group * kBwdGroup + (rg - j * gsize);
+  const int seq = unit / p.heads;
+  const int head = unit - seq * p.heads;
   int row_base = 0, seq_len = p.S;  // first token row and length of this sequence
   if constexpr (VARLEN) {
     row_base = p.cu_seqlens[seq];
