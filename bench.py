@@ -55,6 +55,28 @@ def flops(w):
     return f, 2.5 * f
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of each
+# dominant kernel at the default workload, from the ncu captures summarised in
+# profiles/, with a digest of the kernel sources they were taken on.  Reported
+# only while the sources are unchanged (otherwise null: the counters are stale).
+NCU_TRAFFIC = {
+    "bwd_main": (289_520_896, "d3a9ab0a5972ac6df4f187b59e553c94e4f01612814c5425625e3d06f8f4222c",
+                 ("fa_bwd.cuh", "sm100.cuh")),
+    "fwd": (154_236_416, "2cb36875fb519f2c7dd57447775e13082aa4115f8b5157f56af1f5d33bda1ee3",
+            ("fa_fwd.cuh", "sm100.cuh")),
+}
+
+
+def captured_traffic(kernel: str):
+    import hashlib
+    nbytes, digest, files = NCU_TRAFFIC[kernel]
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "exact_tiled_attention_31_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return nbytes if h.hexdigest() == digest else None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -346,13 +368,14 @@ def main():
 
     # ---- roofline of the dominant kernel
     pk, pk_kind = peaks()
+    traffic = captured_traffic("bwd_main" if ms["bwd_main"] >= ms["fwd"] else "fwd")
     dominant = "bwd_main" if ms["bwd_main"] >= ms["fwd"] else "fwd"
     alg = f_bwd if dominant == "bwd_main" else f_fwd
     achieved = alg / (ms[dominant] * 1e-3) / 1e12
     roofline = {"kernel": "fa::bwd_main_kernel<128,bf16,causal>" if dominant == "bwd_main"
                 else "fa::fwd_kernel<128,bf16,causal,dense>",
                 "bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
                 "peak_source": f"{pk_kind} bf16 dense burst (MEASURED_PEAKS.json bf16_tflops)"
                 if pk_kind == "measured" else "fallback 1590 TFLOP/s (no MEASURED_PEAKS.json)",
                 "algorithmic_flops_per_launch": alg, "ms_per_launch": ms[dominant]}
