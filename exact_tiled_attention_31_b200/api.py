@@ -28,7 +28,7 @@ FA_BF16, FA_FP16 = 0, 1
 
 EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
            "fa_bwd_finish", "fa_bwd_noalloc", "fa_bwd_varlen_workspace_size", "fa_bwd_varlen", "fa_status_string",
-           "fa_check_device_error", "fa_launch_count")
+           "fa_check_device_error", "fa_launch_count", "fa_selftest_timeout")
 
 # Fixed scratch size of fa_bwd_noalloc (FA_BWD_NOALLOC_SCRATCH_BYTES in include/fa.h).
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -77,6 +77,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_check_device_error.argtypes = [vp]
     lib.fa_check_device_error.restype = i
+    lib.fa_selftest_timeout.argtypes = [vp]
+    lib.fa_selftest_timeout.restype = i
     lib.fa_launch_count.argtypes = []
     lib.fa_launch_count.restype = ctypes.c_uint64
     _lib = lib
@@ -141,6 +143,10 @@ def fa_status_string(status: int) -> str:
 
 def fa_check_device_error(stream) -> int:
     return load_library().fa_check_device_error(stream)
+
+
+def fa_selftest_timeout(stream) -> int:
+    return load_library().fa_selftest_timeout(stream)
 
 
 def fa_launch_count() -> int:

@@ -276,6 +276,20 @@ bool ptrs_ok(std::initializer_list<const void*> ps) {
   return true;
 }
 
+// ---------------------------------------------------------------- error-path self-test
+// One warp waits, through the same bounded wait every kernel uses, on an
+// mbarrier that nothing ever arrives on: after the wait limit it records the
+// timeout in the device error word and returns normally.
+__global__ void __launch_bounds__(32) selftest_timeout_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    fa::mbar_init(&bar, 1);
+    fa::fence_mbar_init();
+  }
+  __syncwarp();
+  fa::mbar_wait(&bar, 0, 0x300);
+}
+
 // ---------------------------------------------------------------- allocation-free backward
 // Scratch of fa_bwd_noalloc: a fixed array in device memory, created when
 // the library's module is loaded on a device and held until the process
@@ -443,6 +457,12 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   const fa::BwdParams p = bwd_params(H, nseq, max_seqlen, total, cu_seqlens, D, scale, deterministic != 0,
                                      static_cast<uint8_t*>(workspace), dk, dv);
   return run_bwd(q, k, v, o, dO, lse, dq, p, D, causal != 0, dt == FA_BF16, true, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_selftest_timeout(void* stream) {
+  selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  g_launches.fetch_add(1);
+  return from_cuda(cudaGetLastError());
 }
 
 const char* fa_status_string(fa_status s) {

@@ -202,6 +202,16 @@ const char* fa_status_string(fa_status s);
  */
 fa_status fa_check_device_error(void* stream);
 
+/*
+ * Self-test of the timeout path: launches one warp that waits, with the
+ * library's bounded wait, on a barrier nothing arrives on.  About one second
+ * later it records FA_ERR_TIMEOUT in the device error word and exits normally
+ * (no fault; the context stays usable), so fa_check_device_error(stream)
+ * afterwards returns FA_ERR_TIMEOUT and clears the word.  For tests of callers'
+ * error handling; the pages have no counterpart.
+ */
+fa_status fa_selftest_timeout(void* stream);
+
 /* Number of kernel launches issued by this process through the library so far. */
 uint64_t fa_launch_count(void);
 

@@ -162,3 +162,20 @@ def test_causal_differs_from_full(cuda_device):
     assert (o1.float() - o2.float()).abs().max().item() > 0.1
     # the last row sees every key either way
     torch.testing.assert_close(o1[:, :, -1].float(), o2[:, :, -1].float(), atol=1e-2, rtol=0)
+
+
+def test_timeout_path_reports_and_recovers(cuda_device):
+    """A bounded wait that runs out records FA_ERR_TIMEOUT (no fault, no
+    hang); the error word is cleared by the check and the context keeps
+    working for the next call."""
+    st = torch.cuda.current_stream().cuda_stream
+    assert fa.fa_selftest_timeout(st) == fa.api.FA_OK
+    assert fa.fa_check_device_error(st) == fa.api.FA_ERR_TIMEOUT
+    assert fa.fa_check_device_error(st) == fa.api.FA_OK  # cleared
+    t = inputs.make_dense(1, 2, 256, 64, "bf16", seed=42)
+    d = to_dev(t, cuda_device)
+    o, lse = fa.forward(d["q"], d["k"], d["v"], False, 0.125)
+    fa.check_device_error()
+    o_ref, l_ref = oa.attention_forward(t["q"], t["k"], t["v"], 0.125, False)
+    check_o(o, o_ref, "O after a timeout")
+    check_lse(lse, l_ref, "LSE after a timeout")
