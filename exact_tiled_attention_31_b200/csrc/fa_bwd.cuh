@@ -42,8 +42,8 @@
 //                          per-warp 128-byte-swizzled staging buffer and add it
 //                          to the fp32 accumulator with TMA bulk reductions
 //                          (cp.reduce.async.bulk.tensor .add); under
-//                          deterministic mode instead, key tiles add into query
-//                          tile i one at a time in increasing j.
+//                          deterministic mode the key tiles take turns (in
+//                          increasing j) to issue those reductions for tile i.
 //   bwd_post  dQ = scale * accumulator, rounded to the input dtype.
 // Causal: key tile j only meets query tiles i >= j; only the diagonal tile
 // is masked element-wise.  Packed batches ([H, T, D], cu_seqlens): every
@@ -196,6 +196,9 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, const vo
       "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(src))
       : "memory");
 }
+// Orders this thread's global accesses of the generic proxy with its bulk
+// (async-proxy) operations on global memory.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -552,7 +555,7 @@ __global__ void __launch_bounds__(512, 1)
     const int wq = warp - 12;                        // this warp's 32 rows: 32*wq ..
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     uint8_t* stg = smem + C::STG_OFF + wq * 4096;    // 32 rows x 128 B, 128-B swizzled
-    if (!p.deterministic && lane == 0) tma_prefetch_desc(&tm_dq);
+    if (lane == 0) tma_prefetch_desc(&tm_dq);
     for (int st = 0; st < n_steps; ++st) {
       const int i = i_begin + st;
       if (!__all_sync(0xffffffffu, mbar_wait(dq_full, st & 1, BWD_SITE_DQF))) break;
@@ -564,8 +567,9 @@ __global__ void __launch_bounds__(512, 1)
       for (int cc = 0; cc < D / 32; ++cc) tmem_ld_wait(a[cc]);
       tc_fence_before();
       mbar_arrive(dq_empty);
-      const int q = 128 * i + c;
-      if (!p.deterministic) {
+      // This tile's fp32 partial: TMEM -> per-warp swizzled staging -> TMA bulk
+      // reduce-add into the accumulator, 32 columns at a time.
+      auto reduce_partial = [&]() {
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           if (lane == 0) bulk_wait_read0();  // the previous reduction has read the buffer
@@ -581,37 +585,38 @@ __global__ void __launch_bounds__(512, 1)
             bulk_commit();
           }
         }
+      };
+      if (!p.deterministic) {
+        reduce_partial();
       } else {
-        // key tiles add into query tile i in increasing j: wait for our turn
+        // Key tiles add into query tile i in increasing j: one poller per warp
+        // waits for our turn, the partial goes in with the same bulk
+        // reductions, and the turn passes on only once they have been
+        // performed, so every element sees its additions in one fixed order.
         uint32_t* sem = p.sem + ((size_t)head * p.nseq + seq) * p.n_q + i;
         bool ok = true;
-        if (ld_acquire_gpu(sem) != (uint32_t)j) {
-          const uint64_t t0 = global_ns();
-          while (ld_acquire_gpu(sem) != (uint32_t)j) {
-            if (global_ns() - t0 > kWaitLimitNs) {
-              record_error(DEV_ERR_TIMEOUT, BWD_SITE_SEM);
-              ok = false;
-              break;
+        if (lane == 0) {
+          if (ld_acquire_gpu(sem) != (uint32_t)j) {
+            const uint64_t t0 = global_ns();
+            while (ld_acquire_gpu(sem) != (uint32_t)j) {
+              if (global_ns() - t0 > kWaitLimitNs) {
+                record_error(DEV_ERR_TIMEOUT, BWD_SITE_SEM);
+                ok = false;
+                break;
+              }
             }
           }
+          fence_proxy_async_global();  // our reductions come after the acquire
         }
-        if (ok && q < seq_len) {  // rows of this sequence only
-          float4* dst = reinterpret_cast<float4*>(p.dq_acc + ((size_t)head * p.rows + row_base + q) * D);
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              float4 v = dst[cc * 8 + e];
-              v.x += __uint_as_float(a[cc][4 * e]);
-              v.y += __uint_as_float(a[cc][4 * e + 1]);
-              v.z += __uint_as_float(a[cc][4 * e + 2]);
-              v.w += __uint_as_float(a[cc][4 * e + 3]);
-              dst[cc * 8 + e] = v;
-            }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (ok) {
+          reduce_partial();
+          if (lane == 0) {
+            bulk_wait0();  // this warp's reductions have been performed
+            fence_proxy_async_global();
+          }
         }
-        // every thread's adds are visible device-wide before the counter
-        // moves on (bounded wait on an arrival barrier, no bar.sync)
-        __threadfence();
+        __syncwarp();
         mbar_arrive(dq_done);
         if (c == 0) {
           if (mbar_wait(dq_done, st & 1, BWD_SITE_SEM) && ok) {
