@@ -77,6 +77,25 @@ def captured_traffic(kernel: str):
     return nbytes if h.hexdigest() == digest else None
 
 
+def max_over_ranks(vals: dict, device=None) -> dict:
+    """Per-key maximum over the ranks of the default process group (the
+    slowest rank's time); the values themselves when there is no group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return dict(vals)
+    keys = sorted(vals)
+    t = torch.tensor([float(vals[k]) for k in keys], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return dict(zip(keys, t.tolist()))
+
+
+def job_tflops(world: int, flop_per_rank: float, ms: float) -> float:
+    """Whole-job throughput: every rank runs the same workload (weak scaling),
+    timed by the slowest rank."""
+    return world * flop_per_rank / (ms * 1e-3) / 1e12
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -316,13 +335,10 @@ def main():
     t_step = [e[0].elapsed_time(e[4]) for e in evs]
     ms = {"step": statistics.mean(t_step), "fwd": statistics.mean(t_fwd), "bwd_pre": statistics.mean(t_pre),
           "bwd_main": statistics.mean(t_main), "bwd_finish": statistics.mean(t_fin)}
-    if world > 1:
-        tt = torch.tensor([ms[x] for x in ("step", "fwd", "bwd_pre", "bwd_main", "bwd_finish")], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = dict(zip(("step", "fwd", "bwd_pre", "bwd_main", "bwd_finish"), tt.tolist()))
+    ms = max_over_ranks(ms, device=dev)
     f_fwd, f_bwd = flops(w)
     t_bwd = ms["bwd_pre"] + ms["bwd_main"] + ms["bwd_finish"]
-    value = world * (f_fwd + f_bwd) / (ms["step"] * 1e-3) / 1e12
+    value = job_tflops(world, f_fwd + f_bwd, ms["step"])
     fwd_tf = f_fwd / (ms["fwd"] * 1e-3) / 1e12
     bwd_tf = f_bwd / (t_bwd * 1e-3) / 1e12
     fb_tf = (f_fwd + f_bwd) / ((ms["fwd"] + t_bwd) * 1e-3) / 1e12
@@ -357,12 +373,8 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1) / e_steps
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = tt.item()
-        e2e = {"value": world * (f_fwd + f_bwd) / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks({"e2e": e0.elapsed_time(e1) / e_steps}, device=dev)["e2e"]
+        e2e = {"value": job_tflops(world, f_fwd + f_bwd, e_ms), "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "api": "exact_tiled_attention_31_b200.forward/backward (ctypes over libfa.so)"}
 
