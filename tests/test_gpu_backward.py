@@ -114,3 +114,26 @@ def test_bwd_workspace_reuse_and_dirty(cuda_device):
     for x, y, name in zip(a, b, ("dQ", "dK", "dV")):
         check_grad(y, x, name)
     _check_all(t, True, 0.125, (o, lse, *a), what="dirty workspace")
+
+
+def test_bwd_split_launches_equal_fa_bwd(cuda_device):
+    """fa_bwd_preprocess + fa_bwd_main + fa_bwd_finish (the launches bench.py
+    times one by one) give exactly what fa_bwd gives (deterministic mode)."""
+    B, H, S, D = 1, 3, 520, 128
+    t = inputs.make_dense(B, H, S, D, "bf16", seed=8, with_do=True)
+    d = to_dev(t, cuda_device)
+    o, lse = fa.forward(d["q"], d["k"], d["v"], True, 0.088)
+    ref = fa.backward(d["q"], d["k"], d["v"], o, d["do"], lse, True, 0.088, deterministic=True)
+    nb = fa.fa_bwd_workspace_size(B, H, S, D)
+    ws = torch.empty(nb, dtype=torch.uint8, device=cuda_device)
+    dq, dk, dv = (torch.empty_like(d["q"]) for _ in range(3))
+    st = torch.cuda.current_stream().cuda_stream
+    dt = fa.api.FA_BF16
+    assert fa.fa_bwd_preprocess(o.data_ptr(), d["do"].data_ptr(), lse.data_ptr(), B, H, S, D, dt, ws.data_ptr(), nb,
+                                st) == 0
+    assert fa.fa_bwd_main(d["q"].data_ptr(), d["k"].data_ptr(), d["v"].data_ptr(), d["do"].data_ptr(), dk.data_ptr(),
+                          dv.data_ptr(), B, H, S, D, 0.088, True, dt, True, ws.data_ptr(), nb, st) == 0
+    assert fa.fa_bwd_finish(dq.data_ptr(), B, H, S, D, 0.088, dt, ws.data_ptr(), nb, st) == 0
+    fa.check_device_error()
+    for a, b, name in zip((dq, dk, dv), ref, ("dQ", "dK", "dV")):
+        assert torch.equal(a, b), name
