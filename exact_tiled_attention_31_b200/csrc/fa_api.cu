@@ -64,6 +64,20 @@ bool make_map_f32(CUtensorMap* m, const void* base, int D, long long rows, long 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Per-query rows of the backward's extra K step: bf16 [rows, 16], boxes of
+// 128 rows x 16 columns (32 bytes), 32-byte swizzle.
+bool make_map_cols(CUtensorMap* m, const void* base, long long rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {16, (cuuint64_t)rows, 1};
+  const cuuint64_t strides[2] = {32, (cuuint64_t)rows * 32};
+  const cuuint32_t box[3] = {16, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
@@ -145,20 +159,19 @@ fa_status run_fwd(const void* q, const void* k, const void* v, void* o, float* l
 
 // ---------------------------------------------------------------- backward
 struct WsLayout {
-  size_t dq_acc, lse2, delta, sem, total;
+  size_t dq_acc, cols, sem, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// heads x rows token rows in memory; statistics padded per sequence to
-// ceil(S / 128) * 128 rows (S = the longest sequence)
+// heads x rows token rows in memory; per-query rows (16 bf16 each) padded per
+// sequence to ceil(S / 128) * 128 rows (S = the longest sequence)
 WsLayout ws_layout(long long heads, long long nseq, long long S, long long rows, int D) {
   const long long n_q = (S + 127) / 128, S_pad = n_q * 128;
   WsLayout w;
   w.dq_acc = 0;
-  w.lse2 = up256((size_t)heads * rows * D * 4);
-  w.delta = w.lse2 + up256((size_t)heads * nseq * S_pad * 4);
-  w.sem = w.delta + up256((size_t)heads * nseq * S_pad * 4);
+  w.cols = up256((size_t)heads * rows * D * 4);
+  w.sem = w.cols + up256((size_t)heads * nseq * S_pad * 32);
   w.total = w.sem + up256((size_t)heads * nseq * n_q * 4);
   return w;
 }
@@ -170,8 +183,7 @@ fa::BwdParams bwd_params(int heads, int nseq, int S, int rows, const int* cu, in
   p.dk = dk;
   p.dv = dv;
   p.dq_acc = reinterpret_cast<float*>(ws + w.dq_acc);
-  p.nlse2 = p.nlse2_w = reinterpret_cast<float*>(ws + w.lse2);
-  p.delta = p.delta_w = reinterpret_cast<float*>(ws + w.delta);
+  p.cols = reinterpret_cast<uint16_t*>(ws + w.cols);
   p.sem = reinterpret_cast<uint32_t*>(ws + w.sem);
   p.cu_seqlens = cu;
   p.heads = heads;
@@ -201,7 +213,8 @@ fa_status launch_bwd_pre(const void* o, const void* dO, const float* lse, const 
 
 template <int D, bool BF16, bool CAUSAL, bool VARLEN>
 fa_status launch_bwd_main_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                            const CUtensorMap& mdo, const CUtensorMap& mdq, const fa::BwdParams& p, cudaStream_t st) {
+                            const CUtensorMap& mdo, const CUtensorMap& mdq, const CUtensorMap& mcols,
+                            const fa::BwdParams& p, cudaStream_t st) {
   using C = fa::BwdCfg<D>;
   // groups of kBwdGroup (sequence, head) slices, n_q key tiles each
   const long long units = (long long)p.nseq * p.heads;
@@ -209,7 +222,7 @@ fa_status launch_bwd_main_t(const CUtensorMap& mq, const CUtensorMap& mk, const 
   const long long grid = groups * fa::kBwdGroup * p.n_q;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   if (set_smem<fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN>>(C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
-  fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN><<<(unsigned)grid, 512, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, p);
+  fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN><<<(unsigned)grid, 512, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, mcols, p);
   g_launches.fetch_add(1);
   return from_cuda(cudaGetLastError());
 }
@@ -217,16 +230,17 @@ fa_status launch_bwd_main_t(const CUtensorMap& mq, const CUtensorMap& mk, const 
 template <int D, bool BF16>
 fa_status launch_bwd_main(const void* q, const void* k, const void* v, const void* dO, const fa::BwdParams& p,
                           bool causal, bool varlen, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mdo, mdq;
+  CUtensorMap mq, mk, mv, mdo, mdq, mcols;
   if (!make_map(&mq, q, D, p.rows, p.heads, BF16) || !make_map(&mk, k, D, p.rows, p.heads, BF16) ||
       !make_map(&mv, v, D, p.rows, p.heads, BF16) || !make_map(&mdo, dO, D, p.rows, p.heads, BF16) ||
-      !make_map_f32(&mdq, p.dq_acc, D, p.rows, p.heads))
+      !make_map_f32(&mdq, p.dq_acc, D, p.rows, p.heads) ||
+      !make_map_cols(&mcols, p.cols, (long long)p.heads * p.nseq * p.S_pad))
     return FA_ERR_CUDA;
   if (varlen)
-    return causal ? launch_bwd_main_t<D, BF16, true, true>(mq, mk, mv, mdo, mdq, p, st)
-                  : launch_bwd_main_t<D, BF16, false, true>(mq, mk, mv, mdo, mdq, p, st);
-  return causal ? launch_bwd_main_t<D, BF16, true, false>(mq, mk, mv, mdo, mdq, p, st)
-                : launch_bwd_main_t<D, BF16, false, false>(mq, mk, mv, mdo, mdq, p, st);
+    return causal ? launch_bwd_main_t<D, BF16, true, true>(mq, mk, mv, mdo, mdq, mcols, p, st)
+                  : launch_bwd_main_t<D, BF16, false, true>(mq, mk, mv, mdo, mdq, mcols, p, st);
+  return causal ? launch_bwd_main_t<D, BF16, true, false>(mq, mk, mv, mdo, mdq, mcols, p, st)
+                : launch_bwd_main_t<D, BF16, false, false>(mq, mk, mv, mdo, mdq, mcols, p, st);
 }
 
 template <bool BF16>

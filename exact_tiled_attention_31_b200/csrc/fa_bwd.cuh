@@ -12,9 +12,10 @@
 //     dQ_i  = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i
 //
 // Three launches on the caller's stream:
-//   bwd_pre   D_i = dO_i . O_i (fp32, warp-shuffle reduction), -LSE_i*log2(e)
-//             into a 128-row-padded copy, zero the fp32 dQ accumulator and
-//             the ordering counters.
+//   bwd_pre   D_i = dO_i . O_i (fp32, warp-shuffle reduction); per query row a
+//             16-column bf16 row holding -LSE_i*log2(e) and -D_i, each split
+//             into three bf16 parts (128-row padded); zero the fp32 dQ
+//             accumulator and the ordering counters.
 //   bwd_main  one CTA per 128-row key/value tile j of one head (and, for a
 //             packed batch, one sequence; 512 threads):
 //               warp 0     TMA producer: K_j, V_j once; then Q_i (+ the padded
@@ -61,10 +62,9 @@ struct BwdParams {
   void* dk;                // [heads, rows, D]
   void* dv;                // [heads, rows, D]
   float* dq_acc;           // [heads, rows, D] fp32
-  const float* nlse2;      // [heads, nseq, S_pad]  -LSE * log2(e), -inf in padding rows
-  const float* delta;      // [heads, nseq, S_pad]  D_i, 0 in padding rows
-  float* nlse2_w;          // the same two buffers, written by bwd_pre
-  float* delta_w;
+  uint16_t* cols;          // [heads, nseq, S_pad, 16] bf16 per-query rows (written by bwd_pre):
+                           //   0-8: -LSE*log2(e) in three parts (part k % 3 in column k),
+                           //   9-11: -D_i in three parts, 12-15: 0; padding rows -1e30 and 0
   uint32_t* sem;           // [heads, nseq, n_q] ordering counters (deterministic mode)
   const int* cu_seqlens;   // packed batch only: device int32 [nseq + 1]
   int heads;               // dense: B*H, packed: H
@@ -87,8 +87,9 @@ struct BwdCfg {
   static constexpr uint32_t DO_OFF = 4 * TILE;                   // 1 slot
   static constexpr uint32_t DS_OFF = 5 * TILE;                   // 128 x 128 16-bit, 2 chunks
   static constexpr uint32_t STG_OFF = DS_OFF + 2 * CHUNK;        // 4 warps x (32 rows x 128 B) fp32 staging
-  static constexpr uint32_t STAT_OFF = STG_OFF + 4 * 4096;       // 2 slots x (128 -lse2 + 128 delta) fp32
-  static constexpr uint32_t BAR_OFF = STAT_OFF + 2 * 1024;
+  static constexpr uint32_t CT_OFF = STG_OFF + 4 * 4096;         // 2 slots x per-query rows (128 x 32 B)
+  static constexpr uint32_t ONES_OFF = CT_OFF + 2 * 4096;         // the two constant key-side rows (128 x 32 B)
+  static constexpr uint32_t BAR_OFF = ONES_OFF + 2 * 4096;
   // kv_full q_full[2] q_empty[2] do_full do_empty s_full dp_full p_full ds_full
   // dq_full dq_empty dkv_full drain dq_done
   static constexpr int NBAR = 17;
@@ -148,8 +149,29 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict
 #pragma unroll
     for (int w = G / 2; w > 0; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
     if (in && part == 0) {
-      p.delta_w[row] = valid ? acc : 0.f;
-      p.nlse2_w[row] = valid ? lse[tok] * -1.4426950408889634f : -INFINITY;
+      // per-query row of the extra K step: the tensor core adds
+      // (1/(scale log2 e)) * (-LSE log2 e) to S^T and -D to dP^T
+      const float nl = valid ? lse[tok] * -1.4426950408889634f : -1e30f;
+      const float nd = valid ? -acc : 0.f;
+      float a[3], b[3];
+      a[0] = bf16_round(nl);
+      a[1] = valid ? bf16_round(nl - a[0]) : 0.f;
+      a[2] = valid ? bf16_round(nl - a[0] - a[1]) : 0.f;
+      b[0] = bf16_round(nd);
+      b[1] = bf16_round(nd - b[0]);
+      b[2] = bf16_round(nd - b[0] - b[1]);
+      float v[16];
+#pragma unroll
+      for (int k = 0; k < 9; ++k) v[k] = a[k % 3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) v[9 + k] = b[k];
+#pragma unroll
+      for (int k = 12; k < 16; ++k) v[k] = 0.f;
+      uint4* dst = reinterpret_cast<uint4*>(p.cols + (size_t)row * 16);
+      dst[0] = make_uint4(pack2<true>(v[0], v[1]), pack2<true>(v[2], v[3]), pack2<true>(v[4], v[5]),
+                          pack2<true>(v[6], v[7]));
+      dst[1] = make_uint4(pack2<true>(v[8], v[9]), pack2<true>(v[10], v[11]), pack2<true>(v[12], v[13]),
+                          pack2<true>(v[14], v[15]));
     }
   }
   // zero the dQ accumulator (16-byte stores) and the ordering counters
@@ -177,14 +199,6 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
     r.w = pack2<BF16>(b.z * scale, b.w * scale);
     reinterpret_cast<uint4*>(dq)[i] = r;
   }
-}
-
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
 }
 
 // fp32 tile in shared memory added element-wise into global memory by the
@@ -219,7 +233,8 @@ template <int D, bool BF16, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_cols,
+                    const BwdParams p) {
   using C = BwdCfg<D>;
   // work unit: (key/value tile j, sequence, head).  Blocks walk groups of
   // kBwdGroup (sequence, head) slices; inside a group, ascending j (longest
@@ -265,7 +280,6 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* drain = bars + 14;
   uint64_t* dq_done = bars + 15;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBAR);
-  float* stats = reinterpret_cast<float*>(smem + C::STAT_OFF);
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
@@ -293,6 +307,26 @@ __global__ void __launch_bounds__(512, 1)
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
+  if (threadIdx.x < 256) {
+    // The two constant key-side rows of the extra K step (bf16, 32-byte
+    // swizzle): row set 0 holds 1/(scale log2 e) in three parts (part k / 3 in
+    // column k, k < 9), so against the per-query rows it adds -LSE / scale to
+    // every score; row set 1 holds 1 in columns 9-11, which adds -D to dP.
+    const int set = threadIdx.x >> 7, r = threadIdx.x & 127;
+    const float inv = 1.f / p.scale_log2;
+    const float i0 = bf16_round(inv), i1 = bf16_round(inv - i0), i2 = bf16_round(inv - i0 - i1);
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = set == 0 ? (k < 9 ? (k < 3 ? i0 : k < 6 ? i1 : i2) : 0.f)
+                                                 : ((k >= 9 && k < 12) ? 1.f : 0.f);
+    uint8_t* row = smem + C::ONES_OFF + set * 4096;
+    *reinterpret_cast<uint4*>(row + swz32(r * 32)) =
+        make_uint4(pack2<true>(v[0], v[1]), pack2<true>(v[2], v[3]), pack2<true>(v[4], v[5]), pack2<true>(v[6], v[7]));
+    *reinterpret_cast<uint4*>(row + swz32(r * 32 + 16)) =
+        make_uint4(pack2<true>(v[8], v[9]), pack2<true>(v[10], v[11]), pack2<true>(v[12], v[13]),
+                   pack2<true>(v[14], v[15]));
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -310,6 +344,7 @@ __global__ void __launch_bounds__(512, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_cols);
       mbar_expect_tx(kv_full, 2 * C::TILE);
       for (int c = 0; c < C::CH; ++c) {
         tma_load_3d(smem + C::K_OFF + c * C::CHUNK, &tm_k, kv_full, c * 64, row_base + kv_row0, head);
@@ -322,13 +357,11 @@ __global__ void __launch_bounds__(512, 1)
         // Q_i and its LSE / D rows into Q slot st % 2
         const int qs = st & 1;
         if (st >= 2 && !(ok = mbar_wait(&q_empty[qs], ((st >> 1) - 1) & 1, BWD_SITE_PROD))) break;
-        mbar_expect_tx(&q_full[qs], C::TILE + 1024u);
+        mbar_expect_tx(&q_full[qs], C::TILE + 4096u);
         for (int c = 0; c < C::CH; ++c)
           tma_load_3d(smem + C::Q_OFF + qs * C::TILE + c * C::CHUNK, &tm_q, &q_full[qs], c * 64,
                       row_base + 128 * i, head);
-        const size_t srow = stat_row0 + 128 * i;
-        bulk_load(stats + qs * 256, p.nlse2 + srow, 512, &q_full[qs]);
-        bulk_load(stats + qs * 256 + 128, p.delta + srow, 512, &q_full[qs]);
+        tma_load_3d(smem + C::CT_OFF + qs * 4096, &tm_cols, &q_full[qs], 0, (int)(stat_row0 + 128 * i), 0);
         ++q_issued;
         // dO_i into the dO slot
         if (st >= 1 && !(ok = mbar_wait(do_empty, (st - 1) & 1, BWD_SITE_PROD))) break;
@@ -360,6 +393,10 @@ __global__ void __launch_bounds__(512, 1)
     const uint64_t doK = make_sdesc(smem_addr(smem + C::DO_OFF), 16, 1024);
     const uint64_t doMN = make_sdesc(smem_addr(smem + C::DO_OFF), C::CHUNK, 1024);
     const uint64_t dsMN = make_sdesc(smem_addr(smem + C::DS_OFF), C::CHUNK, 1024);
+    const uint64_t onesL = make_sdesc_sw32(smem_addr(smem + C::ONES_OFF));         // adds -LSE / scale
+    const uint64_t onesD = make_sdesc_sw32(smem_addr(smem + C::ONES_OFF + 4096));  // adds -D
+    const uint64_t ctK = make_sdesc_sw32(smem_addr(smem + C::CT_OFF));              // per-query rows, slot 0
+    constexpr uint32_t ID_AUG = make_idesc(128, 128, true, false, false);           // bf16 x bf16
     // X^T = A_kv B_q^T with both operands K-major (X = S or dP)
     auto kk_product = [&](uint32_t d_col, uint64_t a, uint64_t b) {
 #pragma unroll
@@ -382,9 +419,11 @@ __global__ void __launch_bounds__(512, 1)
                                           mbar_wait(do_full, 0, BWD_SITE_DO));
     if (ok) {
       tc_fence_after();
-      kk_product(C::TM_A, kK, qK);  // S^T(0)
+      kk_product(C::TM_A, kK, qK);  // S^T(0), then - LSE / scale
+      mma_ss_e(tmem + C::TM_A, onesL, ctK, ID_AUG, 1u, e);
       mma_commit_e(s_full, e);
-      kk_product(C::TM_B, vK, doK);  // dP^T(0)
+      kk_product(C::TM_B, vK, doK);  // dP^T(0), then - D
+      mma_ss_e(tmem + C::TM_B, onesD, ctK, ID_AUG, 1u, e);
       mma_commit_e(dp_full, e);
     }
     for (int st = 0; st < n_steps && ok; ++st) {
@@ -401,6 +440,7 @@ __global__ void __launch_bounds__(512, 1)
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&q_full[qs ^ 1], ((st + 1) >> 1) & 1, BWD_SITE_Q)))) break;
         tc_fence_after();
         kk_product(C::TM_A, kK, desc_add(qK, (qs ^ 1) * C::TILE));
+        mma_ss_e(tmem + C::TM_A, onesL, desc_add(ctK, (qs ^ 1) * 4096), ID_AUG, 1u, e);
         mma_commit_e(s_full, e);
       }
       // dK += dS^T Q_i
@@ -419,6 +459,7 @@ __global__ void __launch_bounds__(512, 1)
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(do_full, (st + 1) & 1, BWD_SITE_DO)))) break;
         tc_fence_after();
         kk_product(C::TM_B, vK, doK);
+        mma_ss_e(tmem + C::TM_B, onesD, desc_add(ctK, (qs ^ 1) * 4096), ID_AUG, 1u, e);
         mma_commit_e(dp_full, e);
       }
     }
@@ -449,12 +490,11 @@ __global__ void __launch_bounds__(512, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const float* nl2 = stats + qs * 256;  // -LSE * log2(e) of the 128 queries
-      const float* dlt = nl2 + 128;         // D of the 128 queries
       // visible queries of this key row in tile i: q >= kv under the causal mask
       const int qlo = (CAUSAL && i == j) ? r : 0;
       const bool masked = qlo > 64 * half || !kv_valid;  // some column of this half is invisible
-      // ---- P phase (score columns 64*half .. +63): P^T = 2^(S^T scale log2 e - LSE log2 e)
+      // ---- P phase (score columns 64*half .. +63): the scores already hold
+      // -LSE / scale (extra K step), so P^T = 2^(S'^T scale log2 e)
       uint32_t sv[2][32];
       tmem_ld32(tA + 64 * half, sv[0]);
       tmem_ld32(tA + 64 * half + 32, sv[1]);
@@ -466,9 +506,8 @@ __global__ void __launch_bounds__(512, 1)
       for (int e = 0; e < 32; ++e) {
         const int c = 64 * half + 2 * e;
         const uint32_t* src = sv[e >> 4] + 2 * (e & 15);
-        const float2 nl = *reinterpret_cast<const float2*>(nl2 + c);
         float p0, p1;
-        f2split(ffma2(f2(__uint_as_float(src[0]), __uint_as_float(src[1])), sl2x2, f2(nl.x, nl.y)), p0, p1);
+        f2split(fmul2(f2(__uint_as_float(src[0]), __uint_as_float(src[1])), sl2x2), p0, p1);
         p0 = ex2(p0);
         p1 = ex2(p1);
         if (masked) {
@@ -483,7 +522,8 @@ __global__ void __launch_bounds__(512, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
-      // ---- dS phase: dS^T = P^T (dP^T - D), P as rounded for the products
+      // ---- dS phase: dS^T = P^T (dP^T - D), P as rounded for the products;
+      // dP^T already holds -D (extra K step)
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, st & 1, BWD_SITE_DP));
       if (!ok) break;
       tc_fence_after();
@@ -495,12 +535,9 @@ __global__ void __launch_bounds__(512, 1)
       uint32_t dd[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const int c = 64 * half + 2 * e;
         const uint32_t* src = dv[e >> 4] + 2 * (e & 15);
-        const float2 dl = *reinterpret_cast<const float2*>(dlt + c);
-        const uint64_t dpd = fadd2(f2(__uint_as_float(src[0]), __uint_as_float(src[1])), f2(-dl.x, -dl.y));
         float a, b;
-        f2split(fmul2(widen2<BF16>(pk[e]), dpd), a, b);
+        f2split(fmul2(widen2<BF16>(pk[e]), f2(__uint_as_float(src[0]), __uint_as_float(src[1]))), a, b);
         dd[e] = pack2<BF16>(a, b);
       }
 #pragma unroll

@@ -158,6 +158,13 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uin
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// Descriptor of a K-major operand whose rows are 32 bytes (16 16-bit values,
+// one K step) in the 32-byte swizzle: 8-row groups 256 bytes apart.
+__device__ __forceinline__ uint64_t make_sdesc_sw32(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)(256 >> 4) << 32) | (1ull << 46) |
+         (6ull << 61);
+}
+
 // D(tmem) = A(smem) * B(smem) (+ D if accumulate)
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
@@ -448,5 +455,13 @@ __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
 // rows x 128 B: the 16-byte chunk index is XORed with the row index (the
 // layout TMA writes for CU_TENSOR_MAP_SWIZZLE_128B).
 __device__ __forceinline__ uint32_t swz128(uint32_t off) { return off ^ (((off >> 7) & 7u) << 4); }
+// 32-byte swizzle: 16-byte chunk index (bit 4) XOR bit 7.
+__device__ __forceinline__ uint32_t swz32(uint32_t off) { return off ^ (((off >> 7) & 1u) << 4); }
+// x rounded to the nearest bf16 value, returned as fp32.
+__device__ __forceinline__ float bf16_round(float x) {
+  uint16_t h;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(x));
+  return __uint_as_float((uint32_t)h << 16);
+}
 
 }  // namespace fa

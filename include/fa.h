@@ -91,8 +91,9 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
 
 /*
  * Bytes of device scratch that fa_bwd needs for these sizes: an fp32 dQ
- * accumulator [B, H, S, D], the fp32 row terms D_i = dO_i . O_i [B, H, S],
- * and the ordering counters of deterministic mode, each 256-byte aligned.
+ * accumulator [B, H, S, D], one 32-byte row per query (LSE and the row term
+ * D_i = dO_i . O_i, as bf16 parts, rows padded to multiples of 128), and the
+ * ordering counters of deterministic mode, each 256-byte aligned.
  * Returns 0 for unsupported sizes.
  */
 size_t fa_bwd_workspace_size(int B, int H, int S, int D);
@@ -146,9 +147,10 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
  * The three launches fa_bwd makes, exposed for callers that want to place
  * or time them separately (same arguments, same rules, same workspace; they
  * must run in this order on one stream):
- *   fa_bwd_preprocess  D_i = dO_i . O_i and LSE * log2(e) into the
- *                      workspace; clears the dQ accumulator and the
- *                      deterministic-mode counters.
+ *   fa_bwd_preprocess  D_i = dO_i . O_i and LSE into the workspace (as
+ *                      the per-query rows of an extra product step);
+ *                      clears the dQ accumulator and the deterministic-mode
+ *                      counters.
  *   fa_bwd_main        the tiled pass over key/value tiles: writes dk, dv
  *                      and accumulates unscaled dQ (fp32) in the workspace.
  *   fa_bwd_finish      dq = scale * accumulated dQ, rounded to the dtype.
