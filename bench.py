@@ -57,24 +57,34 @@ def flops(w):
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of each
 # dominant kernel at the default workload, from the ncu captures summarised in
-# profiles/, with a digest of the kernel sources they were taken on.  Reported
-# only while the sources are unchanged (otherwise null: the counters are stale).
+# profiles/, with a digest of the kernel sources (code only) they were taken on.
+# Reported only while that code is unchanged (otherwise null: the counters are stale).
 NCU_TRAFFIC = {
-    "bwd_main": (294_589_440, "7d2810f8d0372e8d6b39c9f0f04b49a53aec9b4acb07a5ec38fc78360db6bd6e",
+    "bwd_main": (294_589_440, "af5197c4e31d9631031a0c99a7e15f94635e740365f46ec943f2ee56522ef679",
                  ("fa_bwd.cuh", "sm100.cuh")),
-    "fwd": (155_227_648, "efa7f805c25dae7da01a94c2a145c9f1ea023d92de79e9d56ab870ccb3baad6a",
+    "fwd": (155_227_648, "bada53d807eda905390c320f5790e8c0d72f7ec6e7f34e324ed5dc10f4acab67",
             ("fa_fwd.cuh", "sm100.cuh")),
 }
 
 
-def captured_traffic(kernel: str):
+def source_digest(files) -> str:
+    """SHA-256 of the kernel sources with comments and blank space removed
+    (edits to comments leave the counters valid; any code change does not)."""
     import hashlib
-    nbytes, digest, files = NCU_TRAFFIC[kernel]
+    import re
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "exact_tiled_attention_31_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
-    return nbytes if h.hexdigest() == digest else None
+        with open(os.path.join(ROOT, "exact_tiled_attention_31_b200", "csrc", f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(re.sub(r"\s+", "", text).encode())
+    return h.hexdigest()
+
+
+def captured_traffic(kernel: str):
+    nbytes, digest, files = NCU_TRAFFIC[kernel]
+    return nbytes if source_digest(files) == digest else None
 
 
 def max_over_ranks(vals: dict, device=None) -> dict:

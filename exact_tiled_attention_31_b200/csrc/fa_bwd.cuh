@@ -18,30 +18,35 @@
 //             accumulator and the ordering counters.
 //   bwd_main  one CTA per 128-row key/value tile j of one head (and, for a
 //             packed batch, one sequence; 512 threads):
-//               warp 0     TMA producer: K_j, V_j once; then Q_i (+ the padded
-//                          LSE/D rows of tile i) into a 2-slot ring and dO_i
-//                          into its own slot.
+//               warp 0     TMA producer: K_j, V_j once; then Q_i (+ the
+//                          per-query rows of tile i) into a 2-slot ring and
+//                          dO_i into its own slot.
 //               warp 1     tcgen05 issuer and TMEM owner.  TMEM columns:
 //                          A = [0,128): S^T, then P^T (16-bit) in [0,64)
 //                          B = [128,256): dP^T, then dS^T in [0,64), then dQ_i
 //                          dV [256,256+D), dK [256+D,256+2D).
 //                          Issue order for query tile i (one step):
 //                            dV  += P^T dO_i          (A = P^T in TMEM)
-//                            S^T(i+1) = K_j Q_{i+1}^T  -> A
+//                            S^T(i+1) = K_j Q_{i+1}^T  -> A, plus one K step
+//                                       that adds -LSE / scale per query
 //                            dK  += dS^T Q_i          (A = dS^T in TMEM)
 //                            dQ_i = dS K_j            (A = dS in smem) -> B
-//                            dP^T(i+1) = V_j dO_{i+1}^T -> B (after dQ_i left TMEM)
+//                            dP^T(i+1) = V_j dO_{i+1}^T -> B (after dQ_i left
+//                                       TMEM), plus one K step that adds -D
 //                          so the exponentials of tile i+1 run while the
 //                          tensor core does dK_i, dQ_i and dP^T(i+1).
-//               warps 4-7  one thread per key row.  P phase: P^T =
-//                          exp2(S^T*scale*log2e - LSE*log2e), kept as 16-bit
+//               warps 4-11 one thread per key row and half of the query
+//                          columns (warps 4-7 queries 0-63, 8-11 queries
+//                          64-127).  P phase: P^T = exp2(S'^T*scale*log2e)
+//                          (S' already holds -LSE/scale), kept as 16-bit
 //                          pairs in registers and written to TMEM A.  dS
-//                          phase: dS^T = P^T (dP^T - D) to TMEM B and, as the
-//                          MN-major A operand of dQ = dS K, to shared memory.
-//                          At the end: dV and scale*dK rows to global memory.
-//               warps 8-11 one thread per query row: move dQ_i from TMEM to a
-//                          per-warp 128-byte-swizzled staging buffer and add it
-//                          to the fp32 accumulator with TMA bulk reductions
+//                          phase: dS^T = P^T dP'^T (dP' already holds -D) to
+//                          TMEM B and, as the MN-major A operand of
+//                          dQ = dS K, to shared memory.  At the end: dV and
+//                          scale*dK rows to global memory.
+//               warps 12-15 one thread per query row: move dQ_i from TMEM to
+//                          a per-warp 128-byte-swizzled staging buffer and add
+//                          it to the fp32 accumulator with TMA bulk reductions
 //                          (cp.reduce.async.bulk.tensor .add); under
 //                          deterministic mode the key tiles take turns (in
 //                          increasing j) to issue those reductions for tile i.
@@ -49,8 +54,8 @@
 // Causal: key tile j only meets query tiles i >= j; only the diagonal tile
 // is masked element-wise.  Packed batches ([H, T, D], cu_seqlens): every
 // sequence is its own problem with tiles counted from its first token; keys
-// past its end get P = 0 and query rows past its end carry LSE padding of
-// -inf, so their dS rows are exactly 0 and nothing leaks into the next
+// past its end get P = 0 and query rows past its end carry a -1e30 score
+// offset (so P = 0) and D = 0, so their dS rows are exactly 0 and nothing leaks into the next
 // sequence's rows (the fp32 reductions of those zero rows add 0).
 #pragma once
 
