@@ -80,3 +80,20 @@ def make_varlen(nseq: int, lo: int, hi: int, H: int, D: int, dtype: str = "bf16"
     if with_do:
         out["do"] = _draw(gen, (H, T, D), 1.0, dt)
     return out
+
+
+def make_decode(B: int, Hq: int, Hkv: int, L: int, D: int, dtype: str = "bf16", seed: int = 42,
+                lo: int = 1) -> dict:
+    """Decode inputs: ``seq_lens`` int32 [B] drawn first, uniform in [lo, L];
+    then q [B, Hq, D] and the caches k, v [B, Hkv, L, D] as fp32 N(0, 1)
+    rounded to ``dtype`` (cache rows past a sequence's length hold values too;
+    they must not be read)."""
+    gen = torch.Generator().manual_seed(seed)
+    lens = torch.randint(lo, L + 1, (B,), generator=gen, dtype=torch.int64)
+    dt = torch_dtype(dtype)
+    return {
+        "seq_lens": lens.to(torch.int32),
+        "q": _draw(gen, (B, Hq, D), 1.0, dt),
+        "k": _draw(gen, (B, Hkv, L, D), 1.0, dt),
+        "v": _draw(gen, (B, Hkv, L, D), 1.0, dt),
+    }

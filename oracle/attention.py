@@ -267,6 +267,58 @@ def varlen_backward(q, k, v, do, cu_seqlens, scale: float, causal: bool, heads=N
     return dq, dk, dv
 
 
+def decode_forward(q, k_cache, v_cache, seq_lens, scale: float):
+    """One new query token per (sequence, query head) against its KV cache.
+
+    ``q`` [B, Hq, D]; ``k_cache``, ``v_cache`` [B, Hkv, L, D] with Hq a
+    multiple of Hkv: query head h reads KV head ``h // (Hq // Hkv)``
+    (grouped-query attention; Hkv = Hq is multi-head, Hkv = 1 multi-query).
+    Sequence b holds ``seq_lens[b]`` valid cached keys.  The new token is the
+    last position, so every cached key is visible and each (b, h) is the plain
+    definition for a single query row.  Returns O [B, Hq, D] and LSE [B, Hq].
+    Decode reads the KV cache once per generated token, with GQA/MQA sharing
+    one KV head among several query heads ("Flash Attention 的算法设计原理",
+    "训练与推理价值" and "练习口述回答").
+    """
+    q, k, v = to_f64(q), to_f64(k_cache), to_f64(v_cache)
+    B, Hq, D = q.shape
+    Hkv = k.shape[1]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    group = Hq // Hkv
+    lens = [int(x) for x in (seq_lens.tolist() if hasattr(seq_lens, "tolist") else seq_lens)]
+    o = np.zeros((B, Hq, v.shape[-1]))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        L = lens[b]
+        for h in range(Hq):
+            kv = h // group
+            ob, lb = _head_forward(q[b, h][None, :], k[b, kv, :L], v[b, kv, :L], scale, False)
+            o[b, h], lse[b, h] = ob[0], lb[0]
+    return o, lse
+
+
+def merge_partials(o_parts, lse_parts):
+    """Combine results of the same query rows over disjoint key subsets.
+
+    ``o_parts`` [S, ..., D] (each normalised over its own subset) and
+    ``lse_parts`` [S, ...]: since exp(LSE_s) is the subset's sum of
+    exponentials, LSE = log sum_s exp(LSE_s) and O = sum_s exp(LSE_s - LSE) O_s
+    (the same rescaling as the running update of "From Self-Attention to
+    FlashAttention", §二, applied once per subset).  Subsets with no key carry
+    LSE = -inf and weight 0.
+    """
+    o_parts, lse_parts = to_f64(o_parts), to_f64(lse_parts)
+    m = lse_parts.max(axis=0)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(lse_parts - m_safe)
+    tot = w.sum(axis=0)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        lse = np.where(tot > 0, m_safe + np.log(tot), -np.inf)
+        o = np.where(tot[..., None] > 0, (w[..., None] * o_parts).sum(axis=0) / tot[..., None], 0.0)
+    return o, lse
+
+
 def flop_count(lengths, heads: int, d: int, causal: bool) -> tuple[float, float]:
     """(forward, backward) FLOPs by the usual convention.
 

@@ -399,3 +399,77 @@ def test_pins_catch_planted_mistakes(name, monkeypatch):
         except (AssertionError, ValueError, IndexError):
             failed.append(pin.__name__)
     assert failed, f"planted mistake {name} passed every pin"
+
+
+# ---------------------------------------------------------------- decode
+def _decode_inputs(B=2, Hq=8, Hkv=2, L=37, D=8, seed=3):
+    g = np.random.default_rng(seed)
+    q = g.standard_normal((B, Hq, D))
+    k = g.standard_normal((B, Hkv, L, D))
+    v = g.standard_normal((B, Hkv, L, D))
+    lens = np.array([L, 5][:B] + [L] * max(0, B - 2))
+    return q, k, v, lens
+
+
+def test_decode_is_the_last_row_of_causal_attention():
+    """A decode step is the last query row of causal attention over the
+    sequence's keys (new token at the end sees every cached key)."""
+    q, k, v, lens = _decode_inputs(B=2, Hq=4, Hkv=4)
+    o, lse = oa.decode_forward(q, k, v, lens, 0.3)
+    for b in range(2):
+        L = lens[b]
+        for h in range(4):
+            qq = np.concatenate([np.zeros((L - 1, q.shape[-1])), q[b, h][None]], axis=0)
+            # brute force: explicit exp/sum over the visible keys of the last row
+            s = [0.3 * float(q[b, h] @ k[b, h, j]) for j in range(L)]
+            mx = max(s)
+            w = [math.exp(x - mx) for x in s]
+            ref = sum(wi * v[b, h, j] for j, wi in enumerate(w)) / sum(w)
+            assert np.allclose(o[b, h], ref, atol=1e-12)
+            assert abs(lse[b, h] - (mx + math.log(sum(w)))) < 1e-12
+            ob, lb = oa.attention_forward(qq, k[b, h, :L], v[b, h, :L], 0.3, True)
+            assert np.allclose(ob[-1], o[b, h], atol=1e-12) and abs(lb[-1] - lse[b, h]) < 1e-12
+
+
+def test_decode_gqa_equals_repeated_kv_heads():
+    q, k, v, lens = _decode_inputs(B=2, Hq=8, Hkv=2)
+    o, lse = oa.decode_forward(q, k, v, lens, 0.25)
+    o2, lse2 = oa.decode_forward(q, np.repeat(k, 4, axis=1), np.repeat(v, 4, axis=1), lens, 0.25)
+    assert np.allclose(o, o2, atol=1e-13) and np.allclose(lse, lse2, atol=1e-13)
+
+
+def test_decode_q_zero_is_mean_of_visible_values():
+    q, k, v, lens = _decode_inputs(B=2, Hq=4, Hkv=1)
+    o, lse = oa.decode_forward(np.zeros_like(q), k, v, lens, 0.5)
+    for b in range(2):
+        assert np.allclose(o[b], v[b, 0, :lens[b]].mean(axis=0), atol=1e-13)
+        assert np.allclose(lse[b], math.log(lens[b]), atol=1e-13)
+
+
+def test_merge_of_split_keys_equals_the_whole():
+    """Splitting the cached keys into disjoint ranges and merging the
+    per-range (O, LSE) gives the unsplit result; an empty range weighs 0."""
+    q, k, v, lens = _decode_inputs(B=1, Hq=2, Hkv=2, L=50)
+    o, lse = oa.decode_forward(q, k, v, lens, 0.4)
+    cuts = [0, 7, 7, 31, 50]  # includes an empty range
+    parts_o, parts_l = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        if b > a:
+            po, pl = oa.decode_forward(q, k[:, :, a:b], v[:, :, a:b], [b - a], 0.4)
+        else:
+            po, pl = np.zeros_like(o), np.full(lse.shape, -np.inf)
+        parts_o.append(po)
+        parts_l.append(pl)
+    mo, ml = oa.merge_partials(np.stack(parts_o), np.stack(parts_l))
+    assert np.allclose(mo, o, atol=1e-13) and np.allclose(ml, lse, atol=1e-13)
+
+
+def test_decode_planted_mistakes_fail():
+    """A decode that reads the wrong KV head, or the keys past seq_lens, is caught."""
+    q, k, v, lens = _decode_inputs(B=2, Hq=8, Hkv=2)
+    o, _ = oa.decode_forward(q, k, v, lens, 0.25)
+    wrong_head = np.concatenate([k[:, 1:], k[:, :1]], axis=1)
+    o_bad, _ = oa.decode_forward(q, wrong_head, v, lens, 0.25)
+    assert not np.allclose(o, o_bad, atol=1e-6)
+    o_all, _ = oa.decode_forward(q, k, v, [k.shape[2]] * 2, 0.25)
+    assert not np.allclose(o[1], o_all[1], atol=1e-6)  # sequence 1 has only 5 valid keys
