@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="b1_h32_s4096_d128_causal")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
     return ap.parse_args()
 
 
@@ -244,6 +245,59 @@ def run_reference(args, rank, world, w):
 
 # ------------------------------------------------------------------ GPU arm
 
+# Decode leg: one new token per (sequence, query head) against full KV caches,
+# grouped-query heads (32 query heads on 8 KV heads), bf16.  Its bound is HBM:
+# the algorithmic bytes are the cache rows read once plus q, O and LSE.
+DECODE = dict(B=8, Hq=32, Hkv=8, L=8192, D=128)
+
+
+def decode_bytes(d) -> int:
+    cache = 2 * d["B"] * d["Hkv"] * d["L"] * d["D"] * 2
+    return cache + 2 * d["B"] * d["Hq"] * d["D"] * 2 + d["B"] * d["Hq"] * 4
+
+
+def decode_leg(fa, inputs, torch, dev, stream, steps: int, warmup: int, flush, hbm_peak: float, peak_kind: str):
+    d = DECODE
+    host = inputs.make_decode(d["B"], d["Hq"], d["Hkv"], d["L"], d["D"], "bf16", seed=42)
+    q, k, v = (host[x].to(dev) for x in ("q", "k", "v"))
+    lens = torch.full((d["B"],), d["L"], dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((d["B"], d["Hq"]), device=dev, dtype=torch.float32)
+    n = fa.fa_decode_num_splits(d["B"], d["Hkv"], d["L"])
+    ws_bytes = fa.fa_decode_workspace_size(d["B"], d["Hq"], n, d["D"])
+    ws = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
+    scale = 1.0 / math.sqrt(d["D"])
+
+    def call():
+        st = fa.fa_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), lens.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          d["B"], d["Hq"], d["Hkv"], d["L"], d["D"], scale, fa.api.FA_BF16, n, ws.data_ptr(),
+                          ws_bytes, stream.cuda_stream)
+        if st != 0:
+            raise fa.FAError(st, "fa_decode")
+
+    for _ in range(max(warmup, 3)):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in evs:
+        flush.zero_()  # the caches (268 MB) exceed L2 anyway; the flush keeps q and O cold too
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    fa.check_device_error()
+    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs)
+    nbytes = decode_bytes(d)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": "decode_b8_hq32_hkv8_l8192_d128_bf16", **d, "n_splits": n, "ms_per_step": ms,
+            "value": gbs, "unit": "GB/s", "tokens_per_s": d["B"] / (ms * 1e-3),
+            "roofline": {"kernel": "fa::decode_split_kernel<128,bf16> + fa::decode_merge_kernel<128,bf16>",
+                         "bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "traffic": None, "algorithmic_bytes_per_launch": nbytes,
+                         "peak_source": f"{peak_kind} copy bandwidth (hbm_gbs)"}}
+
+
 def main():
     args = parse()
     w = WORKLOADS[args.workload]
@@ -408,6 +462,15 @@ def main():
         cpu = {"value": fl / sec / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
                "sample": f"fp64 fwd+bwd of {nh} of {B * H} heads (full S={S}), {sec:.1f} s"}
 
+    decode = None
+    if not args.no_decode:
+        decode = decode_leg(fa, inputs, torch, dev, stream, max(10, min(args.steps, 50)), args.warmup, flush,
+                            pk["hbm_gbs"], pk_kind)
+        d_ms = max_over_ranks({"d": decode["ms_per_step"]}, device=dev)["d"]
+        d_gbs = decode_bytes(DECODE) / (d_ms * 1e-3) / 1e9
+        decode.update(ms_per_step=d_ms, value=d_gbs, tokens_per_s=DECODE["B"] / (d_ms * 1e-3), per="GPU (max over ranks)")
+        decode["roofline"].update(achieved=d_gbs, frac=d_gbs / pk["hbm_gbs"])
+
     clocks = sampler.summary(clock_rows)
     if rank == 0:
         out = {
@@ -422,7 +485,7 @@ def main():
             "fwd_bwd_pct_of_2250": 100 * fb_tf / DATASHEET_TFLOPS,
             "fwd_frac_of_measured": fwd_tf / pk["bf16_tflops"], "bwd_frac_of_measured": bwd_tf / pk["bf16_tflops"],
             "kernel_ms": ms, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches, "clocks": clocks,
+            "gpu_launches": launches, "clocks": clocks, "decode": decode,
         }
         print(json.dumps(out), flush=True)
     if world > 1:

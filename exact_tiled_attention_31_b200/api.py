@@ -28,7 +28,8 @@ FA_BF16, FA_FP16 = 0, 1
 
 EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
            "fa_bwd_finish", "fa_bwd_noalloc", "fa_bwd_varlen_workspace_size", "fa_bwd_varlen", "fa_status_string",
-           "fa_check_device_error", "fa_launch_count", "fa_selftest_timeout")
+           "fa_check_device_error", "fa_launch_count", "fa_selftest_timeout", "fa_decode_num_splits",
+           "fa_decode_workspace_size", "fa_decode")
 
 # Fixed scratch size of fa_bwd_noalloc (FA_BWD_NOALLOC_SCRATCH_BYTES in include/fa.h).
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -79,6 +80,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_check_device_error.restype = i
     lib.fa_selftest_timeout.argtypes = [vp]
     lib.fa_selftest_timeout.restype = i
+    lib.fa_decode_num_splits.argtypes = [i, i, i]
+    lib.fa_decode_num_splits.restype = i
+    lib.fa_decode_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_decode_workspace_size.restype = sz
+    lib.fa_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp]
+    lib.fa_decode.restype = i
     lib.fa_launch_count.argtypes = []
     lib.fa_launch_count.restype = ctypes.c_uint64
     _lib = lib
@@ -135,6 +142,20 @@ def fa_bwd_varlen(q, k, v, o, dO, lse, dq, dk, dv, cu_seqlens, nseq, max_seqlen,
     return load_library().fa_bwd_varlen(q, k, v, o, dO, lse, dq, dk, dv, cu_seqlens, nseq, max_seqlen, total, H, D,
                                         scale, int(causal), dt, int(deterministic), workspace, workspace_bytes,
                                         stream)
+
+
+def fa_decode_num_splits(B, Hkv, L_max) -> int:
+    return load_library().fa_decode_num_splits(B, Hkv, L_max)
+
+
+def fa_decode_workspace_size(B, Hq, n_splits, D) -> int:
+    return load_library().fa_decode_workspace_size(B, Hq, n_splits, D)
+
+
+def fa_decode(q, k_cache, v_cache, seq_lens, o, lse, B, Hq, Hkv, L_max, D, scale, dt, n_splits, workspace,
+              workspace_bytes, stream) -> int:
+    return load_library().fa_decode(q, k_cache, v_cache, seq_lens, o, lse, B, Hq, Hkv, L_max, D, scale, dt, n_splits,
+                                    workspace, workspace_bytes, stream)
 
 
 def fa_status_string(status: int) -> str:
@@ -273,6 +294,37 @@ def backward_noalloc(q, k, v, o, do, lse, dq, dk, dv, causal: bool, scale: float
     if st != FA_OK:
         raise FAError(st, "fa_bwd_noalloc")
     return dq, dk, dv
+
+
+def decode(q, k_cache, v_cache, seq_lens, scale: float | None = None, n_splits: int | None = None, out=None,
+           lse=None, workspace=None, stream=None):
+    """One decode step: q [B, Hq, D] against caches [B, Hkv, L_max, D] holding
+    ``seq_lens`` (CUDA int32 [B]) valid keys each.  Returns O [B, Hq, D] and
+    fp32 LSE [B, Hq].  ``n_splits`` defaults to the library's choice."""
+    import torch
+    B, Hq, D = q.shape
+    _check((q,), q.shape)
+    _check((k_cache, v_cache), k_cache.shape)
+    if k_cache.dtype != q.dtype:
+        raise TypeError("q and the caches must share one dtype")
+    Bk, Hkv, L, Dk = k_cache.shape
+    if Bk != B or Dk != D:
+        raise ValueError(f"cache shape {tuple(k_cache.shape)} does not match q {tuple(q.shape)}")
+    if not seq_lens.is_cuda or seq_lens.dtype != torch.int32 or tuple(seq_lens.shape) != (B,):
+        raise ValueError("seq_lens must be a CUDA int32 tensor of shape [B]")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    n = fa_decode_num_splits(B, Hkv, L) if n_splits is None else int(n_splits)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32) if lse is None else lse
+    need = fa_decode_workspace_size(B, Hq, n, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=q.device, dtype=torch.uint8)
+    st = fa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seq_lens.data_ptr(), o.data_ptr(),
+                   lse.data_ptr(), B, Hq, Hkv, L, D, scale, _dt(q), n, workspace.data_ptr(), workspace.numel(),
+                   _stream(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_decode")
+    return o, lse
 
 
 def check_device_error(stream=None):

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -13,6 +14,7 @@
 
 #include "../../include/fa.h"
 #include "fa_bwd.cuh"
+#include "fa_decode.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -327,6 +329,41 @@ void* noalloc_scratch() {
   return addr[dev];
 }
 
+// ---------------------------------------------------------------- decode
+struct DecWs {
+  size_t lse, total;
+};
+DecWs dec_layout(long long rows, int n_splits, int D) {  // rows = B * Hq
+  const size_t o_bytes = up256((size_t)rows * n_splits * D * 4);
+  return {o_bytes, o_bytes + up256((size_t)rows * n_splits * 4)};
+}
+
+// Split count for B * Hkv cache streams of up to L_max keys: the fewest
+// splits that give about 0.8 x sm_count CTAs (one CTA fills an SM's shared
+// memory), at most 64 and at least 256 keys each.  Longer key ranges per CTA
+// amortise its start-up and the partial-result write; more than one wave only
+// adds those costs (measured on B200 over 1..64 splits for group sizes 1, 4
+// and 16, 1 to 64 sequences and 1K to 32K keys).
+int dec_splits(long long units, int L_max) {
+  if (units <= 0 || L_max <= 0) return 1;
+  const long long tiles = (L_max + 31) / 32, target = (8 * sm_count() + 9) / 10;
+  const long long nmax = std::max(1LL, std::min(64LL, tiles / 8));
+  return (int)std::max(1LL, std::min(nmax, (target + units - 1) / units));
+}
+
+template <int D, bool BF16>
+fa_status launch_decode_t(const fa::DecParams& p, cudaStream_t st) {
+  using C = fa::DecCfg<D>;
+  if (set_smem<fa::decode_split_kernel<D, BF16>>(C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
+  fa::decode_split_kernel<D, BF16><<<dim3(p.n_splits, p.Hkv, p.B), 128, C::SMEM, st>>>(p);
+  g_launches.fetch_add(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return FA_ERR_CUDA;
+  fa::decode_merge_kernel<D, BF16><<<(unsigned)((long long)p.B * p.Hq), D, 0, st>>>(p);
+  g_launches.fetch_add(1);
+  return from_cuda(cudaGetLastError());
+}
+
 }  // namespace
 
 extern "C" {
@@ -471,6 +508,49 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   const fa::BwdParams p = bwd_params(H, nseq, max_seqlen, total, cu_seqlens, D, scale, deterministic != 0,
                                      static_cast<uint8_t*>(workspace), dk, dv);
   return run_bwd(q, k, v, o, dO, lse, dq, p, D, causal != 0, dt == FA_BF16, true, static_cast<cudaStream_t>(stream));
+}
+
+int fa_decode_num_splits(int B, int Hkv, int L_max) {
+  if (B <= 0 || Hkv <= 0 || L_max <= 0) return 1;
+  return dec_splits((long long)B * Hkv, L_max);
+}
+
+size_t fa_decode_workspace_size(int B, int Hq, int n_splits, int D) {
+  if (B <= 0 || Hq <= 0 || n_splits <= 0 || (D != 64 && D != 128)) return 0;
+  return dec_layout((long long)B * Hq, n_splits, D).total;
+}
+
+fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, const int* seq_lens, void* o, float* lse,
+                    int B, int Hq, int Hkv, int L_max, int D, float scale, fa_dtype dt, int n_splits, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || L_max < 0) return FA_ERR_INVALID_ARG;
+  if (dt != FA_BF16 && dt != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || Hq == 0) return FA_OK;
+  if (Hkv == 0 || Hq % Hkv) return FA_ERR_INVALID_ARG;
+  if (Hq / Hkv > 16) return FA_ERR_UNSUPPORTED;
+  if (n_splits < 1 || n_splits > 1024) return FA_ERR_INVALID_ARG;
+  if (B > 65535 || Hkv > 65535 || (long long)B * Hq > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  if (!ptrs_ok({q, k_cache, v_cache, o, lse}) || !seq_lens || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_INVALID_ARG;
+  const DecWs w = dec_layout((long long)B * Hq, n_splits, D);
+  if (workspace_bytes < w.total) return FA_ERR_INVALID_ARG;
+  fa::DecParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = static_cast<const uint16_t*>(k_cache);
+  p.v = static_cast<const uint16_t*>(v_cache);
+  p.seq_lens = seq_lens;
+  p.o_part = reinterpret_cast<float*>(workspace);
+  p.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.lse);
+  p.o = o;
+  p.lse = lse;
+  p.B = B, p.Hq = Hq, p.Hkv = Hkv, p.L = L_max, p.n_splits = n_splits, p.group = Hq / Hkv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 128) return dt == FA_BF16 ? launch_decode_t<128, true>(p, st) : launch_decode_t<128, false>(p, st);
+  return dt == FA_BF16 ? launch_decode_t<64, true>(p, st) : launch_decode_t<64, false>(p, st);
 }
 
 fa_status fa_selftest_timeout(void* stream) {

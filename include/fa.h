@@ -194,6 +194,44 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          int B, int H, int S, int D, float scale, int causal, fa_dtype dt,
                          int deterministic, void* stream);
 
+/*
+ * Decode: one new query token per (sequence, query head) against a KV cache
+ * ("Flash Attention 的算法设计原理", sections "训练与推理价值" and "练习口述回答":
+ * at inference the new token reads the whole, growing cache, and GQA/MQA
+ * share one KV head among several query heads).  For b < B, h < Hq:
+ *
+ *   O[b,h,:]  = softmax(q[b,h,:] . K[b,h/G,j,:] * scale, j < len_b) V[b,h/G,:,:]
+ *   lse[b,h]  = log sum_{j < len_b} exp(q[b,h,:] . K[b,h/G,j,:] * scale)
+ *
+ * with G = Hq / Hkv and len_b = min(max(seq_lens[b], 0), L_max); every cached
+ * key is visible (the new token is the last position).  len_b = 0 gives
+ * O = 0 and lse = -inf.
+ *
+ *   q        [B, Hq, D] 16-bit (dt), contiguous
+ *   k_cache, v_cache  [B, Hkv, L_max, D] 16-bit, contiguous; rows at or past
+ *            len_b are never read
+ *   seq_lens [B] int32 in device memory (4-byte aligned)
+ *   o        [B, Hq, D] 16-bit (dt);  lse [B, Hq] fp32, natural log
+ *   n_splits number of key ranges each cache is cut into (1..1024).  Each
+ *            range is reduced by its own CTA to a normalised partial O and
+ *            its LSE in the workspace, and a second launch merges them:
+ *            LSE = log sum_s exp(LSE_s), O = sum_s exp(LSE_s - LSE) O_s.
+ *            fa_decode_num_splits() returns the library's choice.
+ *   workspace  device memory of at least fa_decode_workspace_size(B, Hq,
+ *            n_splits, D) bytes, 256-byte aligned, owned by the caller; it
+ *            may be reused once the call's work on `stream` has finished.
+ *
+ * Requirements: D = 64 or 128; Hkv >= 1 with Hq a multiple of Hkv
+ * (FA_ERR_INVALID_ARG otherwise) and G = Hq / Hkv <= 16 (FA_ERR_UNSUPPORTED
+ * otherwise); B, Hkv <= 65535; q, k_cache, v_cache, o, lse 16-byte aligned.
+ * B = 0 or Hq = 0 is a no-op.  Two kernel launches on `stream`.
+ */
+int fa_decode_num_splits(int B, int Hkv, int L_max);
+size_t fa_decode_workspace_size(int B, int Hq, int n_splits, int D);
+fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, const int* seq_lens, void* o,
+                    float* lse, int B, int Hq, int Hkv, int L_max, int D, float scale, fa_dtype dt,
+                    int n_splits, void* workspace, size_t workspace_bytes, void* stream);
+
 /* A static, human-readable name for a status code. */
 const char* fa_status_string(fa_status s);
 

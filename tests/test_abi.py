@@ -121,3 +121,39 @@ def test_bwd_varlen_workspace_and_argument_errors(lib):
     assert call(D=80) == fa.api.FA_ERR_UNSUPPORTED
     assert call(scale=-1.0) == fa.api.FA_ERR_INVALID_ARG
     assert call(nseq=0) == fa.api.FA_OK                       # empty pack: nothing to do
+
+
+def test_decode_workspace_splits_and_argument_errors(lib):
+    def up(x):
+        return (x + 255) // 256 * 256
+    for B, Hq, n, D in [(8, 32, 16, 128), (3, 5, 7, 64), (1, 1, 1, 128)]:
+        assert fa.fa_decode_workspace_size(B, Hq, n, D) == up(B * Hq * n * D * 4) + up(B * Hq * n * 4)
+    assert fa.fa_decode_workspace_size(1, 1, 1, 96) == 0
+    assert fa.fa_decode_workspace_size(1, 1, 0, 64) == 0
+    # the library's split choice: 1..64, at least 256 keys per split
+    for B, Hkv, L in [(8, 8, 8192), (1, 1, 100), (1, 8, 32768), (64, 8, 2048), (1, 1, 1 << 20)]:
+        n = fa.fa_decode_num_splits(B, Hkv, L)
+        assert 1 <= n <= 64 and (n == 1 or L >= 256 * n)
+    assert fa.fa_decode_num_splits(0, 8, 1024) == 1
+    A = 1 << 20
+    ws = fa.fa_decode_workspace_size(2, 8, 4, 64)
+
+    def call(**kw):
+        a = dict(q=A, lens=A, B=2, Hq=8, Hkv=2, L=100, D=64, scale=0.125, dt=0, n=4, ws=A, wsb=ws)
+        a.update(kw)
+        return fa.fa_decode(a["q"], A, A, a["lens"], A, A, a["B"], a["Hq"], a["Hkv"], a["L"], a["D"], a["scale"],
+                            a["dt"], a["n"], a["ws"], a["wsb"], None)
+    assert call(Hkv=3) == fa.api.FA_ERR_INVALID_ARG            # Hq not a multiple of Hkv
+    assert call(Hkv=0) == fa.api.FA_ERR_INVALID_ARG
+    assert call(Hq=34, Hkv=2, wsb=1 << 30) == fa.api.FA_ERR_UNSUPPORTED   # group of 17 query heads
+    assert call(D=96) == fa.api.FA_ERR_UNSUPPORTED
+    assert call(n=0) == fa.api.FA_ERR_INVALID_ARG
+    assert call(n=1025) == fa.api.FA_ERR_INVALID_ARG
+    assert call(lens=A + 2) == fa.api.FA_ERR_INVALID_ARG      # misaligned seq_lens
+    assert call(q=A + 8) == fa.api.FA_ERR_INVALID_ARG         # misaligned q
+    assert call(ws=A + 64) == fa.api.FA_ERR_INVALID_ARG       # workspace not 256-byte aligned
+    assert call(wsb=ws - 1) == fa.api.FA_ERR_INVALID_ARG      # workspace too small
+    assert call(scale=0.0) == fa.api.FA_ERR_INVALID_ARG
+    assert call(dt=5) == fa.api.FA_ERR_INVALID_ARG
+    assert call(L=-1) == fa.api.FA_ERR_INVALID_ARG
+    assert call(B=0) == fa.api.FA_OK                          # empty batch: nothing to do
