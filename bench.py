@@ -65,6 +65,9 @@ NCU_TRAFFIC = {
                  ("fa_bwd.cuh", "sm100.cuh")),
     "fwd": (155_227_648, "bada53d807eda905390c320f5790e8c0d72f7ec6e7f34e324ed5dc10f4acab67",
             ("fa_fwd.cuh", "sm100.cuh")),
+    # decode split kernel, B8 Hq32 Hkv8 L8192 D128 bf16, 2 splits (the merge launch is ~0.3 MB)
+    "decode": (272_446_976, "c1fbc38cecaeeab210d140fe3a556f3bc1a3f4d2d1b54a558dc03779c1023e2d",
+               ("fa_decode.cuh", "sm100.cuh")),
 }
 
 
@@ -256,34 +259,41 @@ def decode_bytes(d) -> int:
     return cache + 2 * d["B"] * d["Hq"] * d["D"] * 2 + d["B"] * d["Hq"] * 4
 
 
-def decode_leg(fa, inputs, torch, dev, stream, steps: int, warmup: int, flush, hbm_peak: float, peak_kind: str):
+def decode_leg(fa, inputs, torch, dev, stream, steps: int, warmup: int, hbm_peak: float, peak_kind: str):
+    """Mean device time of fa_decode (split + merge launches) on DECODE.
+
+    Two sets of inputs (2 x 268 MB of caches, each set above the 126 MB L2)
+    alternate between steps, so a step never finds the previous step's cache
+    rows in L2; no write-flush runs in between (its dirty lines would be
+    written back during the next step and bill it for unrelated traffic)."""
     d = DECODE
-    host = inputs.make_decode(d["B"], d["Hq"], d["Hkv"], d["L"], d["D"], "bf16", seed=42)
-    q, k, v = (host[x].to(dev) for x in ("q", "k", "v"))
+    sets = []
+    for seed in (42, 43):
+        host = inputs.make_decode(d["B"], d["Hq"], d["Hkv"], d["L"], d["D"], "bf16", seed=seed)
+        sets.append(tuple(host[x].to(dev) for x in ("q", "k", "v")))
     lens = torch.full((d["B"],), d["L"], dtype=torch.int32, device=dev)
-    o = torch.empty_like(q)
+    o = torch.empty_like(sets[0][0])
     lse = torch.empty((d["B"], d["Hq"]), device=dev, dtype=torch.float32)
     n = fa.fa_decode_num_splits(d["B"], d["Hkv"], d["L"])
     ws_bytes = fa.fa_decode_workspace_size(d["B"], d["Hq"], n, d["D"])
     ws = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
     scale = 1.0 / math.sqrt(d["D"])
 
-    def call():
+    def call(i):
+        q, k, v = sets[i % 2]
         st = fa.fa_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), lens.data_ptr(), o.data_ptr(), lse.data_ptr(),
                           d["B"], d["Hq"], d["Hkv"], d["L"], d["D"], scale, fa.api.FA_BF16, n, ws.data_ptr(),
                           ws_bytes, stream.cuda_stream)
         if st != 0:
             raise fa.FAError(st, "fa_decode")
 
-    for _ in range(max(warmup, 3)):
-        flush.zero_()
-        call()
+    for i in range(max(warmup, 3)):
+        call(i)
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for e0, e1 in evs:
-        flush.zero_()  # the caches (268 MB) exceed L2 anyway; the flush keeps q and O cold too
+    for i, (e0, e1) in enumerate(evs):
         e0.record(stream)
-        call()
+        call(i)
         e1.record(stream)
     torch.cuda.synchronize()
     fa.check_device_error()
@@ -292,9 +302,12 @@ def decode_leg(fa, inputs, torch, dev, stream, steps: int, warmup: int, flush, h
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"workload": "decode_b8_hq32_hkv8_l8192_d128_bf16", **d, "n_splits": n, "ms_per_step": ms,
             "value": gbs, "unit": "GB/s", "tokens_per_s": d["B"] / (ms * 1e-3),
-            "roofline": {"kernel": "fa::decode_split_kernel<128,bf16> + fa::decode_merge_kernel<128,bf16>",
+            "l2": "two input sets of 268 MB alternate (inputs larger than L2), no flush",
+            "roofline": {"kernel": "fa::decode_split_kernel<128,bf16>" + (
+                             " (2..4-CTA clusters, merged in-kernel)" if 2 <= n <= 4 else
+                             "" if n == 1 else " + fa::decode_merge_kernel<128,bf16>"),
                          "bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
-                         "traffic": None, "algorithmic_bytes_per_launch": nbytes,
+                         "traffic": captured_traffic("decode"), "algorithmic_bytes_per_launch": nbytes,
                          "peak_source": f"{peak_kind} copy bandwidth (hbm_gbs)"}}
 
 
@@ -464,7 +477,8 @@ def main():
 
     decode = None
     if not args.no_decode:
-        decode = decode_leg(fa, inputs, torch, dev, stream, max(10, min(args.steps, 50)), args.warmup, flush,
+        del flush
+        decode = decode_leg(fa, inputs, torch, dev, stream, max(10, min(args.steps, 50)), args.warmup,
                             pk["hbm_gbs"], pk_kind)
         d_ms = max_over_ranks({"d": decode["ms_per_step"]}, device=dev)["d"]
         d_gbs = decode_bytes(DECODE) / (d_ms * 1e-3) / 1e9

@@ -351,17 +351,62 @@ int dec_splits(long long units, int L_max) {
   return (int)std::max(1LL, std::min(nmax, (target + units - 1) / units));
 }
 
+// Clusters of 2 to 4 CTAs merge in-kernel when all CTAs fit in one wave.
+// Larger clusters, or several waves of them, measured slower on B200 than
+// the separate merge launch: a cluster of 197 KB CTAs needs that many free
+// SMs of one GPC at once, and its CTAs wait for its slowest one.
+constexpr int kDecClusterMax = 4;
+
 template <int D, bool BF16>
 fa_status launch_decode_t(const fa::DecParams& p, cudaStream_t st) {
   using C = fa::DecCfg<D>;
+  // caches as [B * Hkv, L, D]; 32-row boxes (L < 32 means no whole tile, so
+  // the box is never used and only has to be valid)
+  CUtensorMap mk, mv;
+  const long long heads = (long long)p.B * p.Hkv;
+  const int rows = std::max(p.L, 1);
+  const unsigned box = (unsigned)std::min(C::KT, rows);
+  if (!make_map(&mk, p.k, D, rows, heads, BF16, box) || !make_map(&mv, p.v, D, rows, heads, BF16, box))
+    return FA_ERR_CUDA;
   if (set_smem<fa::decode_split_kernel<D, BF16>>(C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
-  fa::decode_split_kernel<D, BF16><<<dim3(p.n_splits, p.Hkv, p.B), 128, C::SMEM, st>>>(p);
+  cudaError_t e;
+  const long long ctas = (long long)p.n_splits * p.Hkv * p.B;
+  if (p.n_splits >= 2 && p.n_splits <= kDecClusterMax && ctas <= sm_count()) {
+    // the splits of one (sequence, KV head) as one cluster, merged in-kernel
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.n_splits, p.Hkv, p.B);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.n_splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, fa::decode_split_kernel<D, BF16>, mk, mv, p);
+    g_launches.fetch_add(1);
+    return from_cuda(e);
+  }
+  fa::decode_split_kernel<D, BF16><<<dim3(p.n_splits, p.Hkv, p.B), 128, C::SMEM, st>>>(mk, mv, p);
   g_launches.fetch_add(1);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return FA_ERR_CUDA;
-  fa::decode_merge_kernel<D, BF16><<<(unsigned)((long long)p.B * p.Hq), D, 0, st>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.n_splits == 1) return from_cuda(e);  // one split writes O and LSE itself
+  // the merge as a programmatic dependent launch: it is scheduled while the
+  // split kernel runs and waits (griddepcontrol.wait) for its results
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((long long)p.B * p.Hq));
+  cfg.blockDim = dim3(D);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, fa::decode_merge_kernel<D, BF16>, p);
   g_launches.fetch_add(1);
-  return from_cuda(cudaGetLastError());
+  return from_cuda(e);
 }
 
 }  // namespace

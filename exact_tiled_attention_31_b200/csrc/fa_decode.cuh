@@ -13,12 +13,20 @@
 //
 // B200 mapping.  The work is a stream of the cache through the SMs, bounded by
 // HBM bandwidth, so the cache is split along its length: one CTA per
-// (split, KV head, sequence) covers a contiguous key range and writes a
-// partial result normalised over that range plus its log-sum-exp;
-// decode_merge_kernel then combines the splits (the merge of disjoint key
-// subsets: LSE = log sum exp(LSE_s), O = sum exp(LSE_s - LSE) O_s).
-// Inside a CTA, 4 warps take alternate 32-key tiles, each with its own
-// double-buffered cp.async copy of K and V; the G query rows of the group
+// (split, KV head, sequence) covers a contiguous key range, and the ranges
+// are combined by the merge of disjoint key subsets (LSE = log sum
+// exp(LSE_s), O = sum exp(LSE_s - LSE) O_s).  When the launch runs the
+// splits of one (sequence, KV head) as one thread-block cluster (the host
+// does so for 2 to 4 splits that fit in one wave), rank 0 merges the others'
+// parts through distributed shared memory at the end; with one split the CTA
+// writes O and LSE itself; otherwise each CTA writes a normalised partial O
+// and its LSE and decode_merge_kernel combines them.
+// Inside a CTA, 4 warps take alternate 32-key tiles, each warp with its own
+// ring of stages that its lane 0 fills by TMA (K and V tiles of 32 rows x
+// 64 columns, 128-byte swizzle, completion counted on the stage's mbarrier).
+// A tile that runs past the sequence's last key is copied row by row with
+// cp.async instead, zero-filling the rows past the end, so no cache row at
+// or past the length is ever read.  The G query rows of the group
 // (padded to 16) are the M dimension of m16n8k16 tensor-core products
 // (S = Q K^T, then O += P V with P in registers), which are far from the
 // bound here: 32 KB of K/V per 32-key tile per warp against two products of
@@ -45,17 +53,25 @@ struct DecParams {
 template <int D>
 struct DecCfg {
   static constexpr int KT = 32;                          // keys per warp tile
-  static constexpr int PITCH = D * 2 + 16;               // bytes per cached row in shared memory
-  static constexpr int TILE = KT * PITCH;                // one K or V tile
+  static constexpr int HALF = KT * 128;                  // 32 rows x 64 columns, 128-byte swizzled
+  static constexpr int TILE = KT * D * 2;                // one K or V tile (D / 64 halves)
   static constexpr int WARPS = 4;
-  static constexpr int STAGES = D == 128 ? 3 : 5;        // K+V tiles in flight per warp: STAGES - 1
+  static constexpr int STAGES = D == 128 ? 3 : 6;        // K+V tiles in flight per warp: STAGES - 1
   static constexpr int WARP_BYTES = 2 * STAGES * TILE;
-  static constexpr int SMEM = WARPS * WARP_BYTES;        // D = 128: 208896 bytes, D = 64: 184320
+  static constexpr int SMEM = WARPS * WARP_BYTES + 1024; // + alignment slack; D = 128: 197632 bytes
   static constexpr int CHUNKS = KT * D * 2 / 16;         // 16-byte pieces per tile
   static constexpr int SCRATCH = 3 * 16 + 16 * D;        // floats per warp for the final merge
-  static_assert(SMEM <= 227 * 1024, "shared memory per block");
-  static_assert(WARPS * SCRATCH * 4 <= SMEM, "merge scratch fits in the tile buffers");
+  static_assert(SMEM <= 227 * 1024 - WARPS * STAGES * 8, "shared memory per block");
+  static_assert((WARPS + 1) * SCRATCH * 4 <= WARPS * WARP_BYTES, "merge scratch fits in the tile buffers");
 };
+
+enum : uint32_t { DEC_SITE_KV = 0x300, DEC_SITE_DRAIN = 0x301 };
+
+// byte offset of (row, 8-column chunk c8 of D / 8) in a K or V tile
+template <int D>
+__device__ __forceinline__ uint32_t dec_off(int row, int c8) {
+  return (c8 >> 3) * DecCfg<D>::HALF + row * 128 + (((c8 & 7) ^ (row & 7)) << 4);
+}
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)),
@@ -71,6 +87,40 @@ __device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r
 }
 __device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t& r0, uint32_t& r1) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
+// thread-block cluster: rank, size, barrier, and loads from a peer CTA's
+// shared memory (distributed shared memory)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_addr(p)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ float ld_dsmem(uint32_t a) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_dsmem4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(a)
+               : "memory");
+  return v;
 }
 
 // c[4] += a[4] (16 x 16, row) * b[2] (16 x 8, col), fp32 accumulate
@@ -92,9 +142,13 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(128, 1) decode_split_kernel(const DecParams p) {
+__global__ void __launch_bounds__(128, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        const DecParams p) {
   using C = DecCfg<D>;
-  extern __shared__ __align__(16) uint8_t dsm[];
+  extern __shared__ uint8_t dsm_raw[];
+  __shared__ uint64_t bars[C::WARPS][C::STAGES];
+  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int len = min(max(p.seq_lens[b], 0), p.L);
@@ -102,6 +156,19 @@ __global__ void __launch_bounds__(128, 1) decode_split_kernel(const DecParams p)
   const int per = ((len + p.n_splits - 1) / p.n_splits + C::KT - 1) / C::KT * C::KT;
   const int start = split * per, end = min(len, start + per);
   const int n_tiles = end > start ? (end - start + C::KT - 1) / C::KT : 0;
+  const int bh = b * p.Hkv + kvh;  // cache head index (third tensor-map coordinate)
+  if (lane == 0) {
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(&bars[warp][s], 1);
+    fence_mbar_init();
+  }
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  // the merge launch may start once every block has got here; it still waits
+  // for this grid's completion before reading the partial results
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __syncwarp();
 
   // Q as the A operand (rows = the group's query heads, padded to 16 with zeros)
   const int r0 = lane >> 2, r1 = r0 + 8, cq = 2 * (lane & 3);
@@ -119,29 +186,41 @@ __global__ void __launch_bounds__(128, 1) decode_split_kernel(const DecParams p)
 
   uint8_t* kbuf = dsm + warp * C::WARP_BYTES;  // K tiles [STAGES], then V tiles [STAGES]
   uint8_t* vbuf = kbuf + C::STAGES * C::TILE;
-  const uint16_t* kh = p.k + ((size_t)b * p.Hkv + kvh) * p.L * D;
-  const uint16_t* vh = p.v + ((size_t)b * p.Hkv + kvh) * p.L * D;
-  // the warp's i-th tile is tile warp + WARPS * i of the split, in stage
-  // i % STAGES.  One commit group per call (empty past the warp's last tile)
-  // keeps the wait_group counts uniform; keys past `end` are zero-filled.
+  const uint16_t* kh = p.k + (size_t)bh * p.L * D;
+  const uint16_t* vh = p.v + (size_t)bh * p.L * D;
+  // The warp's i-th tile is tile warp + WARPS * i of the split, in stage
+  // i % STAGES.  A whole tile comes by TMA; the one tile that runs past
+  // `end` (always the split's last, so the warp's last) by cp.async with
+  // the rows past `end` zero-filled.
+  auto full_tile = [&](int i) { return start + C::KT * (warp + C::WARPS * i) + C::KT <= end; };
   auto issue = [&](int i) {
     const int t = warp + C::WARPS * i;
-    if (t < n_tiles) {
-      const int key0 = start + C::KT * t;
-      uint8_t* kd = kbuf + (i % C::STAGES) * C::TILE;
-      uint8_t* vd = vbuf + (i % C::STAGES) * C::TILE;
+    if (t >= n_tiles) return;
+    const int key0 = start + C::KT * t, s = i % C::STAGES;
+    uint8_t* kd = kbuf + s * C::TILE;
+    uint8_t* vd = vbuf + s * C::TILE;
+    if (key0 + C::KT <= end) {
+      if (lane == 0) {
+        mbar_expect_tx(&bars[warp][s], 2 * C::TILE);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_3d(kd + h * C::HALF, &tm_k, &bars[warp][s], 64 * h, key0, bh);
+          tma_load_3d(vd + h * C::HALF, &tm_v, &bars[warp][s], 64 * h, key0, bh);
+        }
+      }
+    } else {
 #pragma unroll
       for (int j = 0; j < C::CHUNKS / 32; ++j) {
         const int c = lane + 32 * j;
-        const int row = c / (D * 2 / 16), col = c % (D * 2 / 16);
+        const int row = c / (D / 8), c8 = c % (D / 8);
         const int key = key0 + row;
         const bool in = key < end;
-        const size_t off = (size_t)(in ? key : 0) * D + col * 8;
-        cp_async16(kd + row * C::PITCH + col * 16, kh + off, in ? 16u : 0u);
-        cp_async16(vd + row * C::PITCH + col * 16, vh + off, in ? 16u : 0u);
+        const size_t off = (size_t)(in ? key : 0) * D + c8 * 8;
+        cp_async16(kd + dec_off<D>(row, c8), kh + off, in ? 16u : 0u);
+        cp_async16(vd + dec_off<D>(row, c8), vh + off, in ? 16u : 0u);
       }
+      cp_async_commit();
     }
-    cp_async_commit();
   };
 
   float oacc[D / 8][4];
@@ -155,9 +234,18 @@ __global__ void __launch_bounds__(128, 1) decode_split_kernel(const DecParams p)
   for (int i = 0; i < C::STAGES - 1; ++i) issue(i);
   for (int i = 0; i < my_tiles; ++i) {
     issue(i + C::STAGES - 1);
-    cp_async_wait<C::STAGES - 1>();  // the warp's tile i has landed (own copies)
-    __syncwarp();                    // ... and every lane's copies are visible
     const int t = warp + C::WARPS * i, st = i % C::STAGES;
+    if (full_tile(i)) {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[warp][st], (i / C::STAGES) & 1, DEC_SITE_KV));
+      if (!ok) {  // error recorded: let the warp's copies in flight land (bounded), then stop
+        for (int j = i + 1; j < min(i + C::STAGES, my_tiles); ++j)
+          if (full_tile(j)) mbar_wait(&bars[warp][j % C::STAGES], (j / C::STAGES) & 1, DEC_SITE_DRAIN);
+        break;
+      }
+    } else {
+      cp_async_wait<0>();
+      __syncwarp();
+    }
     const uint32_t ks = smem_addr(kbuf + st * C::TILE), vs = smem_addr(vbuf + st * C::TILE);
     // S = Q K^T: 16 rows x 32 keys (4 tiles of 8)
     float sacc[4][4];
@@ -168,7 +256,7 @@ __global__ void __launch_bounds__(128, 1) decode_split_kernel(const DecParams p)
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt) {
         uint32_t b0, b1;
-        ldsm_x2(ks + (8 * nt + (lane & 7)) * C::PITCH + (16 * kk + 8 * ((lane >> 3) & 1)) * 2, b0, b1);
+        ldsm_x2(ks + dec_off<D>(8 * nt + (lane & 7), 2 * kk + ((lane >> 3) & 1)), b0, b1);
         mma16816<BF16>(sacc[nt], qa[kk], b0, b1);
       }
     }
@@ -226,12 +314,13 @@ __global__ void __launch_bounds__(128, 1) decode_split_kernel(const DecParams p)
 #pragma unroll
       for (int n = 0; n < D / 8; ++n) {
         uint32_t b0, b1;
-        ldsm_x2_trans(vs + (16 * k2 + (lane & 15)) * C::PITCH + 8 * n * 2, b0, b1);
+        ldsm_x2_trans(vs + dec_off<D>(16 * k2 + (lane & 15), n), b0, b1);
         mma16816<BF16>(oacc[n], pa[k2], b0, b1);
       }
     }
-    __syncwarp();  // every lane is done with this buffer before it is refilled
+    __syncwarp();  // every lane is done with this stage before it is refilled
   }
+  cp_async_wait<0>();
 
   // the lane's shares of the row sums -> the row's (4 lanes of a quad)
 #pragma unroll
@@ -260,17 +349,17 @@ __global__ void __launch_bounds__(128, 1) decode_split_kernel(const DecParams p)
     ws[48 + r1 * D + 8 * n + cq + 1] = oacc[n][3];
   }
   __syncthreads();
-  // thread -> (row, 16 of the D columns)
+  // thread -> (row, 16 of the D columns): this CTA's (max, sums, unnormalised O)
   constexpr int PARTS = D / 16;
   const int row = threadIdx.x / PARTS, part = threadIdx.x % PARTS;
-  if (row < p.group && threadIdx.x < 16 * PARTS) {
+  const bool active = row < p.group && threadIdx.x < 16 * PARTS;
+  float mm = -INFINITY, lt = 0.f, lrt = 0.f, acc[16];
+#pragma unroll
+  for (int d = 0; d < 16; ++d) acc[d] = 0.f;
+  if (active) {
     const float* w0 = reinterpret_cast<const float*>(dsm);
-    float mm = -INFINITY;
 #pragma unroll
     for (int w = 0; w < C::WARPS; ++w) mm = fmaxf(mm, w0[w * C::SCRATCH + row]);
-    float lt = 0.f, lrt = 0.f, acc[16];
-#pragma unroll
-    for (int d = 0; d < 16; ++d) acc[d] = 0.f;
 #pragma unroll
     for (int w = 0; w < C::WARPS; ++w) {
       const float* wp = w0 + w * C::SCRATCH;
@@ -280,20 +369,90 @@ __global__ void __launch_bounds__(128, 1) decode_split_kernel(const DecParams p)
 #pragma unroll
       for (int d = 0; d < 16; ++d) acc[d] += wp[48 + row * D + 16 * part + d] * sc;
     }
-    const size_t orow = ((size_t)b * p.Hq + kvh * p.group + row) * p.n_splits + split;
-    const float inv = lrt > 0.f ? 1.f / lrt : 0.f;
-    float4* dst = reinterpret_cast<float4*>(p.o_part + orow * D + 16 * part);
+  }
+  const size_t qrow = (size_t)b * p.Hq + kvh * p.group + row;
+
+  if (cluster_nctarank() > 1) {
+    // The splits of this (sequence, KV head) form one cluster: each CTA
+    // publishes its part in its own shared memory and rank 0 merges them
+    // through distributed shared memory, the same rescaling as between warps.
+    float* pub = reinterpret_cast<float*>(dsm) + C::WARPS * C::SCRATCH;  // m[16] l[16] lr[16] O[16][D]
+    if (active) {
+      if (part == 0) {
+        pub[row] = mm;
+        pub[16 + row] = lt;
+        pub[32 + row] = lrt;
+      }
 #pragma unroll
-    for (int d = 0; d < 4; ++d)
-      dst[d] = make_float4(acc[4 * d] * inv, acc[4 * d + 1] * inv, acc[4 * d + 2] * inv, acc[4 * d + 3] * inv);
-    if (part == 0) p.lse_part[orow] = lt > 0.f ? (mm + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
+      for (int d = 0; d < 16; ++d) pub[48 + row * D + 16 * part + d] = acc[d];
+    }
+    cluster_sync();  // every part is published
+    if (cluster_ctarank() == 0 && active) {
+      const uint32_t nct = cluster_nctarank();
+      float M = -INFINITY;
+      for (uint32_t r = 0; r < nct; ++r) M = fmaxf(M, ld_dsmem(dsmem_addr(pub + row, r)));
+      float L = 0.f, LR = 0.f, O[16];
+#pragma unroll
+      for (int d = 0; d < 16; ++d) O[d] = 0.f;
+      for (uint32_t r = 0; r < nct; ++r) {
+        const float mr = ld_dsmem(dsmem_addr(pub + row, r));
+        const float w = M == -INFINITY ? 0.f : ex2(mr - M);
+        L += w * ld_dsmem(dsmem_addr(pub + 16 + row, r));
+        LR += w * ld_dsmem(dsmem_addr(pub + 32 + row, r));
+        const uint32_t oa = dsmem_addr(pub + 48 + row * D + 16 * part, r);
+#pragma unroll
+        for (int d = 0; d < 4; ++d) {
+          const float4 v = ld_dsmem4(oa + 16 * d);
+          O[4 * d] += w * v.x;
+          O[4 * d + 1] += w * v.y;
+          O[4 * d + 2] += w * v.z;
+          O[4 * d + 3] += w * v.w;
+        }
+      }
+      const float inv = LR > 0.f ? 1.f / LR : 0.f;
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + qrow * D + 16 * part);
+#pragma unroll
+      for (int d = 0; d < 2; ++d)
+        dst[d] = make_uint4(pack2<BF16>(O[8 * d] * inv, O[8 * d + 1] * inv),
+                            pack2<BF16>(O[8 * d + 2] * inv, O[8 * d + 3] * inv),
+                            pack2<BF16>(O[8 * d + 4] * inv, O[8 * d + 5] * inv),
+                            pack2<BF16>(O[8 * d + 6] * inv, O[8 * d + 7] * inv));
+      if (part == 0) p.lse[qrow] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+    }
+    cluster_sync();  // rank 0 has read every peer before any CTA exits
+    return;
+  }
+
+  if (active) {
+    const float inv = lrt > 0.f ? 1.f / lrt : 0.f;
+    const float lse = lt > 0.f ? (mm + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
+    if (p.n_splits == 1) {  // the split is the whole cache: final O and LSE
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + qrow * D + 16 * part);
+#pragma unroll
+      for (int d = 0; d < 2; ++d)
+        dst[d] = make_uint4(pack2<BF16>(acc[8 * d] * inv, acc[8 * d + 1] * inv),
+                            pack2<BF16>(acc[8 * d + 2] * inv, acc[8 * d + 3] * inv),
+                            pack2<BF16>(acc[8 * d + 4] * inv, acc[8 * d + 5] * inv),
+                            pack2<BF16>(acc[8 * d + 6] * inv, acc[8 * d + 7] * inv));
+      if (part == 0) p.lse[qrow] = lse;
+    } else {  // partial result for decode_merge_kernel
+      const size_t orow = qrow * p.n_splits + split;
+      float4* dst = reinterpret_cast<float4*>(p.o_part + orow * D + 16 * part);
+#pragma unroll
+      for (int d = 0; d < 4; ++d)
+        dst[d] = make_float4(acc[4 * d] * inv, acc[4 * d + 1] * inv, acc[4 * d + 2] * inv, acc[4 * d + 3] * inv);
+      if (part == 0) p.lse_part[orow] = lse;
+    }
   }
 }
 
 // O and LSE of each (sequence, query head) from its splits: LSE = log sum
 // exp(LSE_s), O = sum exp(LSE_s - LSE) O_s.  One block of D threads per row.
+// Launched as a programmatic dependent of decode_split_kernel: its blocks may
+// be resident before the split kernel ends and wait here for its results.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(D) decode_merge_kernel(const DecParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const size_t row = blockIdx.x;  // b * Hq + h
   const float* lp = p.lse_part + row * p.n_splits;
   float mx = -INFINITY;
