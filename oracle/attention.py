@@ -70,6 +70,13 @@ __all__ = [
     "attention_forward_online",
     "varlen_forward",
     "varlen_backward",
+    "decode_forward",
+    "merge_partials",
+    "philox4x32_10",
+    "dropout_keep_threshold",
+    "dropout_keep",
+    "attention_forward_dropout",
+    "attention_backward_dropout",
     "flop_count",
 ]
 
@@ -317,6 +324,123 @@ def merge_partials(o_parts, lse_parts):
         lse = np.where(tot > 0, m_safe + np.log(tot), -np.inf)
         o = np.where(tot[..., None] > 0, (w[..., None] * o_parts).sum(axis=0) / tot[..., None], 0.0)
     return o, lse
+
+
+# ---------------------------------------------------------------- dropout
+#
+# Dropout on the attention probabilities, the branch the pages ask to be
+# tested on its own ("Flash Attention 的算法设计原理", "练习口述回答": dropout is
+# one of the paths to cover separately; the mask has to be regenerated in the
+# backward rather than stored, which needs a counter-based generator).  The
+# pages fix neither the generator nor where the mask sits, so the reading is:
+#
+# * P is the exact softmax; the output uses  Pd = P * M / (1 - p)  with
+#   M_ij in {0, 1} kept with probability 1 - p;  O = Pd V.  LSE is the
+#   statistic of the undropped softmax (dropout comes after normalisation).
+# * M_ij for head bh (= b * H + h), query i, key j is decided by one output
+#   word of Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random
+#   numbers: as easy as 1, 2, 3", SC 2011) with
+#       counter = (j >> 1, i >> 1, bh, offset mod 2^32),
+#       key     = (seed mod 2^32, seed >> 32 mod 2^32),
+#   word number 2 * (i & 1) + (j & 1); the element is kept when that word is
+#   below  floor((1 - p) * 2^32).  One call covers a 2 x 2 block of (query,
+#   key), so it is as cheap to regenerate by key rows as by query rows.
+# * Backward of L = sum(dO * O) with the same M:
+#       dV = Pd^T dO,  dPd = dO V^T,  dP = dPd * M / (1 - p),
+#       D_i = sum_j P_ij dP_ij  (= dO_i . O_i),  dS = P * (dP - D),
+#       dQ = scale dS K,  dK = scale dS^T Q.
+
+_MASK32 = np.uint64(0xFFFFFFFF)
+_PHILOX_M = (np.uint64(0xD2511F53), np.uint64(0xCD9E8D57))   # round multipliers
+_PHILOX_W = (np.uint64(0x9E3779B9), np.uint64(0xBB67AE85))   # key schedule increments
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32 with 10 rounds on broadcastable uint32 counter words.
+
+    ``ctr`` is four arrays (c0, c1, c2, c3), ``key`` two integers (k0, k1).
+    Each round multiplies c0 and c2 by the two round constants, keeps the
+    64-bit products' halves, and mixes them with c1, c3 and the round key:
+    (c0, c1, c2, c3) <- (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1,
+    lo(M0 c0)); the key advances by the Weyl increments between rounds.
+    Returns the four output words as uint32 arrays.
+    """
+    c = [np.asarray(x).astype(np.uint64) & _MASK32 for x in ctr]
+    c = np.broadcast_arrays(*c)
+    k0, k1 = np.uint64(int(key[0]) & 0xFFFFFFFF), np.uint64(int(key[1]) & 0xFFFFFFFF)
+    for r in range(10):
+        if r:
+            k0 = (k0 + _PHILOX_W[0]) & _MASK32
+            k1 = (k1 + _PHILOX_W[1]) & _MASK32
+        p0 = c[0] * _PHILOX_M[0]   # < 2^64: exact in uint64
+        p1 = c[2] * _PHILOX_M[1]
+        c = [(p1 >> np.uint64(32)) ^ c[1] ^ k0, p1 & _MASK32, (p0 >> np.uint64(32)) ^ c[3] ^ k1, p0 & _MASK32]
+    return [x.astype(np.uint32) for x in c]
+
+
+def dropout_keep_threshold(p: float) -> int:
+    """Integer threshold floor((1 - p) 2^32): a word below it keeps the element."""
+    if not 0.0 <= p < 1.0:
+        raise ValueError("dropout probability must be in [0, 1)")
+    return int(np.floor((1.0 - p) * 4294967296.0))
+
+
+def dropout_keep(bh: int, rows, cols, p: float, seed: int, offset: int) -> np.ndarray:
+    """Boolean keep mask [len(rows), len(cols)] of head bh (query rows, key columns)."""
+    i = np.asarray(rows, dtype=np.int64)[:, None]
+    j = np.asarray(cols, dtype=np.int64)[None, :]
+    words = philox4x32_10((j >> 1, i >> 1, bh, offset & 0xFFFFFFFF), (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF))
+    sel = 2 * (i & 1) + (j & 1)
+    w = np.choose(np.broadcast_to(sel, np.broadcast_shapes(i.shape, j.shape)), words)
+    return w.astype(np.int64) < dropout_keep_threshold(p)
+
+
+def _head_dropout(q, k, v, do, scale, causal, p, keep):
+    s = attention_scores(q, k, scale)
+    pr, m, l = _three_pass(s, _visible(q.shape[0], k.shape[0], causal))
+    pd = pr * keep / (1.0 - p)
+    o = pd @ v
+    with np.errstate(divide="ignore"):
+        lse = np.where(l > 0, m + np.log(l), -np.inf)
+    if do is None:
+        return o, lse
+    dv = pd.T @ do
+    dp = (do @ v.T) * keep / (1.0 - p)
+    d_row = (pr * dp).sum(axis=1)
+    ds = pr * (dp - d_row[:, None])
+    return scale * (ds @ k), scale * (ds.T @ q), dv
+
+
+def attention_forward_dropout(q, k, v, scale: float, causal: bool, p: float, seed: int, offset: int, heads=None):
+    """O, LSE with dropout on P for [B, H, S, D] inputs (LSE of the undropped softmax)."""
+    q, k, v = to_f64(q), to_f64(k), to_f64(v)
+    B, H, S, D = q.shape
+    pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else list(heads)
+    o = np.zeros((len(pairs), S, v.shape[-1]))
+    lse = np.zeros((len(pairs), S))
+    for n, (b, h) in enumerate(pairs):
+        keep = dropout_keep(b * H + h, np.arange(S), np.arange(S), p, seed, offset)
+        o[n], lse[n] = _head_dropout(q[b, h], k[b, h], v[b, h], None, scale, causal, p, keep)
+    if heads is None:
+        return o.reshape(B, H, S, -1), lse.reshape(B, H, S)
+    return o, lse
+
+
+def attention_backward_dropout(q, k, v, do, scale: float, causal: bool, p: float, seed: int, offset: int,
+                               heads=None):
+    """dQ, dK, dV of L = sum(dO * O) with the dropout mask of the forward."""
+    q, k, v, do = to_f64(q), to_f64(k), to_f64(v), to_f64(do)
+    B, H, S, D = q.shape
+    pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else list(heads)
+    out = [np.zeros((len(pairs), S, D)) for _ in range(2)] + [np.zeros((len(pairs), S, v.shape[-1]))]
+    for n, (b, h) in enumerate(pairs):
+        keep = dropout_keep(b * H + h, np.arange(S), np.arange(S), p, seed, offset)
+        g = _head_dropout(q[b, h], k[b, h], v[b, h], do[b, h], scale, causal, p, keep)
+        for t, x in zip(out, g):
+            t[n] = x
+    if heads is None:
+        return tuple(t.reshape(B, H, S, -1) for t in out)
+    return tuple(out)
 
 
 def flop_count(lengths, heads: int, d: int, causal: bool) -> tuple[float, float]:
