@@ -29,7 +29,7 @@ FA_BF16, FA_FP16 = 0, 1
 EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
            "fa_bwd_finish", "fa_bwd_noalloc", "fa_bwd_varlen_workspace_size", "fa_bwd_varlen", "fa_status_string",
            "fa_check_device_error", "fa_launch_count", "fa_selftest_timeout", "fa_decode_num_splits",
-           "fa_decode_workspace_size", "fa_decode")
+           "fa_decode_workspace_size", "fa_decode", "fa_fwd_dropout", "fa_bwd_dropout")
 
 # Fixed scratch size of fa_bwd_noalloc (FA_BWD_NOALLOC_SCRATCH_BYTES in include/fa.h).
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -86,6 +86,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_decode_workspace_size.restype = sz
     lib.fa_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp]
     lib.fa_decode.restype = i
+    u64 = ctypes.c_uint64
+    lib.fa_fwd_dropout.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, f, u64, u64, vp]
+    lib.fa_fwd_dropout.restype = i
+    lib.fa_bwd_dropout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, f, u64, u64, vp, sz, vp]
+    lib.fa_bwd_dropout.restype = i
     lib.fa_launch_count.argtypes = []
     lib.fa_launch_count.restype = ctypes.c_uint64
     _lib = lib
@@ -142,6 +147,18 @@ def fa_bwd_varlen(q, k, v, o, dO, lse, dq, dk, dv, cu_seqlens, nseq, max_seqlen,
     return load_library().fa_bwd_varlen(q, k, v, o, dO, lse, dq, dk, dv, cu_seqlens, nseq, max_seqlen, total, H, D,
                                         scale, int(causal), dt, int(deterministic), workspace, workspace_bytes,
                                         stream)
+
+
+def fa_fwd_dropout(q, k, v, o, lse, B, H, S, D, scale, causal, dt, dropout_p, seed, offset, stream) -> int:
+    return load_library().fa_fwd_dropout(q, k, v, o, lse, B, H, S, D, scale, int(causal), dt, dropout_p, seed, offset,
+                                         stream)
+
+
+def fa_bwd_dropout(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, causal, dt, deterministic, dropout_p, seed,
+                   offset, workspace, workspace_bytes, stream) -> int:
+    return load_library().fa_bwd_dropout(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, int(causal), dt,
+                                         int(deterministic), dropout_p, seed, offset, workspace, workspace_bytes,
+                                         stream)
 
 
 def fa_decode_num_splits(B, Hkv, L_max) -> int:
@@ -204,14 +221,22 @@ def _stream(stream):
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def forward(q, k, v, causal: bool, scale: float | None = None, out=None, lse=None, stream=None):
-    """O, LSE of [B, H, S, D] inputs; LSE is fp32 [B, H, S]."""
+def forward(q, k, v, causal: bool, scale: float | None = None, out=None, lse=None, stream=None,
+            dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
+    """O, LSE of [B, H, S, D] inputs; LSE is fp32 [B, H, S].  ``dropout_p`` > 0
+    drops attention probabilities with the counter-based mask of (seed, offset)."""
     import torch
     B, H, S, D = q.shape
     _check((q, k, v), q.shape)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     o = torch.empty_like(q) if out is None else out
     lse = torch.empty((B, H, S), device=q.device, dtype=torch.float32) if lse is None else lse
+    if dropout_p:
+        st = fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, S, D,
+                            scale, causal, _dt(q), float(dropout_p), int(seed), int(offset), _stream(stream))
+        if st != FA_OK:
+            raise FAError(st, "fa_fwd_dropout")
+        return o, lse
     st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, S, D, scale,
                 causal, _dt(q), _stream(stream))
     if st != FA_OK:
@@ -239,8 +264,9 @@ def forward_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool, scale: fl
 
 
 def backward(q, k, v, o, do, lse, causal: bool, scale: float | None = None, deterministic: bool = False,
-             workspace=None, stream=None):
-    """dQ, dK, dV of [B, H, S, D] inputs given the forward's O and LSE."""
+             workspace=None, stream=None, dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
+    """dQ, dK, dV of [B, H, S, D] inputs given the forward's O and LSE (and
+    the forward's dropout_p, seed and offset, if it dropped)."""
     import torch
     B, H, S, D = q.shape
     _check((q, k, v, o, do), q.shape)
@@ -249,6 +275,14 @@ def backward(q, k, v, o, do, lse, causal: bool, scale: float | None = None, dete
     nbytes = fa_bwd_workspace_size(B, H, S, D)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(max(nbytes, 1), device=q.device, dtype=torch.uint8)
+    if dropout_p:
+        st = fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, S, D, scale, causal, _dt(q),
+                            deterministic, float(dropout_p), int(seed), int(offset), workspace.data_ptr(),
+                            workspace.numel(), _stream(stream))
+        if st != FA_OK:
+            raise FAError(st, "fa_bwd_dropout")
+        return dq, dk, dv
     st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
                 dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, S, D, scale, causal, _dt(q), deterministic,
                 workspace.data_ptr(), workspace.numel(), _stream(stream))

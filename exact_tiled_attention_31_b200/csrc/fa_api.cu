@@ -109,12 +109,12 @@ int sm_count() {
 fa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
 
 // ---------------------------------------------------------------- forward
-template <int D, bool BF16, bool CAUSAL, bool VARLEN>
+template <int D, bool BF16, bool CAUSAL, bool VARLEN, bool DROPOUT = false>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
                      cudaStream_t st) {
   using C = fa::FwdCfg<D>;
-  auto kern = fa::fwd_kernel<D, BF16, CAUSAL, VARLEN>;
-  cudaError_t e = set_smem<fa::fwd_kernel<D, BF16, CAUSAL, VARLEN>>(C::SMEM);
+  auto kern = fa::fwd_kernel<D, BF16, CAUSAL, VARLEN, DROPOUT>;
+  cudaError_t e = set_smem<fa::fwd_kernel<D, BF16, CAUSAL, VARLEN, DROPOUT>>(C::SMEM);
   if (e != cudaSuccess) return FA_ERR_CUDA;
   const long long grid = (long long)p.n_pairs * p.nseq * p.heads;
   if (grid <= 0) return FA_OK;
@@ -125,8 +125,11 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 }
 
 template <int D, bool BF16>
-fa_status dispatch_fwd(bool causal, bool varlen, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const fa::FwdParams& p, cudaStream_t st) {
+fa_status dispatch_fwd(bool causal, bool varlen, bool dropout, const CUtensorMap& mq, const CUtensorMap& mk,
+                       const CUtensorMap& mv, const fa::FwdParams& p, cudaStream_t st) {
+  if (dropout)  // dense batches only
+    return causal ? launch_fwd<D, BF16, true, false, true>(mq, mk, mv, p, st)
+                  : launch_fwd<D, BF16, false, false, true>(mq, mk, mv, p, st);
   if (varlen)
     return causal ? launch_fwd<D, BF16, true, true>(mq, mk, mv, p, st)
                   : launch_fwd<D, BF16, false, true>(mq, mk, mv, p, st);
@@ -136,7 +139,7 @@ fa_status dispatch_fwd(bool causal, bool varlen, const CUtensorMap& mq, const CU
 
 fa_status run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu, int heads,
                   int seqlen, long long rows, int nseq, int D, float scale, bool causal, bool bf16, bool varlen,
-                  cudaStream_t st) {
+                  cudaStream_t st, const fa::Dropout* drop = nullptr) {
   // query and key/value tiles of 128 rows
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, D, rows, heads, bf16, 128) || !make_map(&mk, k, D, rows, heads, bf16, 128) ||
@@ -152,11 +155,13 @@ fa_status run_fwd(const void* q, const void* k, const void* v, void* o, float* l
   p.nseq = nseq;
   p.n_pairs = (seqlen + 255) / 256;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.drop = drop ? *drop : fa::Dropout{};
+  const bool dr = drop != nullptr;
   if (D == 64)
-    return bf16 ? dispatch_fwd<64, true>(causal, varlen, mq, mk, mv, p, st)
-                : dispatch_fwd<64, false>(causal, varlen, mq, mk, mv, p, st);
-  return bf16 ? dispatch_fwd<128, true>(causal, varlen, mq, mk, mv, p, st)
-              : dispatch_fwd<128, false>(causal, varlen, mq, mk, mv, p, st);
+    return bf16 ? dispatch_fwd<64, true>(causal, varlen, dr, mq, mk, mv, p, st)
+                : dispatch_fwd<64, false>(causal, varlen, dr, mq, mk, mv, p, st);
+  return bf16 ? dispatch_fwd<128, true>(causal, varlen, dr, mq, mk, mv, p, st)
+              : dispatch_fwd<128, false>(causal, varlen, dr, mq, mk, mv, p, st);
 }
 
 // ---------------------------------------------------------------- backward
@@ -197,6 +202,7 @@ fa::BwdParams bwd_params(int heads, int nseq, int S, int rows, const int* cu, in
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.deterministic = deterministic;
+  p.drop = fa::Dropout{};
   return p;
 }
 
@@ -213,7 +219,7 @@ fa_status launch_bwd_pre(const void* o, const void* dO, const float* lse, const 
   return from_cuda(cudaGetLastError());
 }
 
-template <int D, bool BF16, bool CAUSAL, bool VARLEN>
+template <int D, bool BF16, bool CAUSAL, bool VARLEN, bool DROPOUT = false>
 fa_status launch_bwd_main_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const CUtensorMap& mdo, const CUtensorMap& mdq, const CUtensorMap& mcols,
                             const fa::BwdParams& p, cudaStream_t st) {
@@ -223,21 +229,25 @@ fa_status launch_bwd_main_t(const CUtensorMap& mq, const CUtensorMap& mk, const 
   const long long groups = (units + fa::kBwdGroup - 1) / fa::kBwdGroup;
   const long long grid = groups * fa::kBwdGroup * p.n_q;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-  if (set_smem<fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN>>(C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
-  fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN><<<(unsigned)grid, 512, C::SMEM, st>>>(mq, mk, mv, mdo, mdq, mcols, p);
+  if (set_smem<fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN, DROPOUT>>(C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
+  fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN, DROPOUT><<<(unsigned)grid, 512, C::SMEM, st>>>(mq, mk, mv, mdo, mdq,
+                                                                                           mcols, p);
   g_launches.fetch_add(1);
   return from_cuda(cudaGetLastError());
 }
 
 template <int D, bool BF16>
 fa_status launch_bwd_main(const void* q, const void* k, const void* v, const void* dO, const fa::BwdParams& p,
-                          bool causal, bool varlen, cudaStream_t st) {
+                          bool causal, bool varlen, bool dropout, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mdo, mdq, mcols;
   if (!make_map(&mq, q, D, p.rows, p.heads, BF16) || !make_map(&mk, k, D, p.rows, p.heads, BF16) ||
       !make_map(&mv, v, D, p.rows, p.heads, BF16) || !make_map(&mdo, dO, D, p.rows, p.heads, BF16) ||
       !make_map_f32(&mdq, p.dq_acc, D, p.rows, p.heads) ||
       !make_map_cols(&mcols, p.cols, (long long)p.heads * p.nseq * p.S_pad))
     return FA_ERR_CUDA;
+  if (dropout)  // dense batches only
+    return causal ? launch_bwd_main_t<D, BF16, true, false, true>(mq, mk, mv, mdo, mdq, mcols, p, st)
+                  : launch_bwd_main_t<D, BF16, false, false, true>(mq, mk, mv, mdo, mdq, mcols, p, st);
   if (varlen)
     return causal ? launch_bwd_main_t<D, BF16, true, true>(mq, mk, mv, mdo, mdq, mcols, p, st)
                   : launch_bwd_main_t<D, BF16, false, true>(mq, mk, mv, mdo, mdq, mcols, p, st);
@@ -255,7 +265,8 @@ fa_status launch_bwd_post(void* dq, const fa::BwdParams& p, int D, cudaStream_t 
 
 // The three backward launches over prepared parameters (dense or packed).
 fa_status run_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
-                  void* dq, const fa::BwdParams& p, int D, bool causal, bool bf16, bool varlen, cudaStream_t st) {
+                  void* dq, const fa::BwdParams& p, int D, bool causal, bool bf16, bool varlen, cudaStream_t st,
+                  bool dropout = false) {
   fa_status c;
   if (D == 64)
     c = bf16 ? launch_bwd_pre<64, true>(o, dO, lse, p, varlen, st) : launch_bwd_pre<64, false>(o, dO, lse, p, varlen, st);
@@ -264,11 +275,11 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* o, co
              : launch_bwd_pre<128, false>(o, dO, lse, p, varlen, st);
   if (c != FA_OK) return c;
   if (D == 64)
-    c = bf16 ? launch_bwd_main<64, true>(q, k, v, dO, p, causal, varlen, st)
-             : launch_bwd_main<64, false>(q, k, v, dO, p, causal, varlen, st);
+    c = bf16 ? launch_bwd_main<64, true>(q, k, v, dO, p, causal, varlen, dropout, st)
+             : launch_bwd_main<64, false>(q, k, v, dO, p, causal, varlen, dropout, st);
   else
-    c = bf16 ? launch_bwd_main<128, true>(q, k, v, dO, p, causal, varlen, st)
-             : launch_bwd_main<128, false>(q, k, v, dO, p, causal, varlen, st);
+    c = bf16 ? launch_bwd_main<128, true>(q, k, v, dO, p, causal, varlen, dropout, st)
+             : launch_bwd_main<128, false>(q, k, v, dO, p, causal, varlen, dropout, st);
   if (c != FA_OK) return c;
   return bf16 ? launch_bwd_post<true>(dq, p, D, st) : launch_bwd_post<false>(dq, p, D, st);
 }
@@ -409,6 +420,21 @@ fa_status launch_decode_t(const fa::DecParams& p, cudaStream_t st) {
   return from_cuda(e);
 }
 
+// ---------------------------------------------------------------- dropout
+// Keep threshold floor((1 - p) 2^32) and scale 1 / (1 - p); p in (0, 1).
+fa::Dropout make_dropout(float p, uint64_t seed, uint64_t offset) {
+  fa::Dropout d;
+  const double keep = 1.0 - (double)p;
+  d.thresh = (uint32_t)std::min(std::floor(keep * 4294967296.0), 4294967295.0);
+  d.seed_lo = (uint32_t)seed;
+  d.seed_hi = (uint32_t)(seed >> 32);
+  d.offset = (uint32_t)offset;
+  d.scale = (float)(1.0 / keep);
+  return d;
+}
+
+bool dropout_p_ok(float p) { return std::isfinite(p) && p >= 0.f && p < 1.f; }
+
 }  // namespace
 
 extern "C" {
@@ -478,10 +504,10 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* d
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool cz = causal != 0;
   if (D == 64)
-    return dt == FA_BF16 ? launch_bwd_main<64, true>(q, k, v, dO, p, cz, false, st)
-                         : launch_bwd_main<64, false>(q, k, v, dO, p, cz, false, st);
-  return dt == FA_BF16 ? launch_bwd_main<128, true>(q, k, v, dO, p, cz, false, st)
-                       : launch_bwd_main<128, false>(q, k, v, dO, p, cz, false, st);
+    return dt == FA_BF16 ? launch_bwd_main<64, true>(q, k, v, dO, p, cz, false, false, st)
+                         : launch_bwd_main<64, false>(q, k, v, dO, p, cz, false, false, st);
+  return dt == FA_BF16 ? launch_bwd_main<128, true>(q, k, v, dO, p, cz, false, false, st)
+                       : launch_bwd_main<128, false>(q, k, v, dO, p, cz, false, false, st);
 }
 
 fa_status fa_bwd_finish(void* dq, int B, int H, int S, int D, float scale, fa_dtype dt, void* workspace,
@@ -511,6 +537,44 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                   stream);
   if (c != FA_OK) return c;
   return fa_bwd_finish(dq, B, H, S, D, scale, dt, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S,
+                         int D, float scale, int causal, fa_dtype dt, float dropout_p, uint64_t seed,
+                         uint64_t offset, void* stream) {
+  if (!dropout_p_ok(dropout_p)) return FA_ERR_INVALID_ARG;
+  if (dropout_p == 0.f) return fa_fwd(q, k, v, o, lse, B, H, S, D, scale, causal, dt, stream);
+  if (B < 0 || H < 0 || S < 0) return FA_ERR_INVALID_ARG;
+  if (dt != FA_BF16 && dt != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || S == 0) return FA_OK;
+  if (!ptrs_ok({q, k, v, o, lse})) return FA_ERR_INVALID_ARG;
+  const long long heads = (long long)B * H;
+  if (heads > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  const fa::Dropout d = make_dropout(dropout_p, seed, offset);
+  return run_fwd(q, k, v, o, lse, nullptr, (int)heads, S, S, 1, D, scale, causal != 0, dt == FA_BF16, false,
+                 static_cast<cudaStream_t>(stream), &d);
+}
+
+fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                         void* dq, void* dk, void* dv, int B, int H, int S, int D, float scale, int causal,
+                         fa_dtype dt, int deterministic, float dropout_p, uint64_t seed, uint64_t offset,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (!dropout_p_ok(dropout_p)) return FA_ERR_INVALID_ARG;
+  if (dropout_p == 0.f)
+    return fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, causal, dt, deterministic, workspace,
+                  workspace_bytes, stream);
+  fa_status c = bwd_common_checks(B, H, S, D, dt, workspace, workspace_bytes);
+  if (c != FA_OK) return c;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || S == 0) return FA_OK;
+  if (!ptrs_ok({q, k, v, o, dO, lse, dq, dk, dv})) return FA_ERR_INVALID_ARG;
+  fa::BwdParams p = bwd_params(B * H, 1, S, S, nullptr, D, scale, deterministic != 0,
+                               static_cast<uint8_t*>(workspace), dk, dv);
+  p.drop = make_dropout(dropout_p, seed, offset);
+  return run_bwd(q, k, v, o, dO, lse, dq, p, D, causal != 0, dt == FA_BF16, false, static_cast<cudaStream_t>(stream),
+                 true);
 }
 
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,

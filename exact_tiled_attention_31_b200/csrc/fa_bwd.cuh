@@ -79,6 +79,7 @@ struct BwdParams {
   int S_pad, n_q;          // ceil(S / 128) * 128, ceil(S / 128)
   float scale, scale_log2;
   int deterministic;
+  Dropout drop;            // DROPOUT instances only
 };
 
 template <int D>
@@ -234,7 +235,7 @@ __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
 // ---------------------------------------------------------------------------
 // bwd_main
 // ---------------------------------------------------------------------------
-template <int D, bool BF16, bool CAUSAL, bool VARLEN>
+template <int D, bool BF16, bool CAUSAL, bool VARLEN, bool DROPOUT = false>
 __global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -521,9 +522,43 @@ __global__ void __launch_bounds__(512, 1)
         }
         pk[e] = pack2<BF16>(p0, p1);
       }
+      // dropout keep masks of the 64 query columns: bit e of keep_lo / keep_hi
+      // for queries 2e and 2e + 1 of this half.  One Philox call covers query
+      // pair e x key rows (2m, 2m + 1), which sit in one lane pair: the even
+      // lane draws pairs 0-15, the odd lane 16-31, and each hands the other
+      // key row's two words across.
+      uint32_t keep_lo = 0xFFFFFFFFu, keep_hi = 0xFFFFFFFFu;
+      if constexpr (DROPOUT) {
+        const bool odd = (lane & 1u) != 0;
+        const uint32_t th = p.drop.thresh;
+        const uint32_t keypair = (uint32_t)kv >> 1, qp0 = (uint32_t)(128 * i + 64 * half) >> 1;
+        keep_lo = keep_hi = 0u;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const uint4 w = philox4x32_10(make_uint4(keypair, qp0 + k + (odd ? 16u : 0u), (uint32_t)head, p.drop.offset),
+                                        p.drop.seed_lo, p.drop.seed_hi);
+          // word 2 * (query & 1) + (key & 1)
+          const uint32_t own0 = odd ? w.y : w.x, own1 = odd ? w.w : w.z;  // this key row
+          const uint32_t oth0 = odd ? w.x : w.y, oth1 = odd ? w.z : w.w;  // the partner key row
+          const uint32_t got0 = __shfl_xor_sync(0xffffffffu, oth0, 1), got1 = __shfl_xor_sync(0xffffffffu, oth1, 1);
+          const uint32_t a0 = odd ? got0 : own0, a1 = odd ? got1 : own1;  // query pair k
+          const uint32_t b0 = odd ? own0 : got0, b1 = odd ? own1 : got1;  // query pair 16 + k
+          keep_lo |= (a0 < th ? 1u : 0u) << k | (b0 < th ? 1u : 0u) << (16 + k);
+          keep_hi |= (a1 < th ? 1u : 0u) << k | (b1 < th ? 1u : 0u) << (16 + k);
+        }
+      }
       // P^T pairs go to columns [64*half, 64*half + 32) of A (inside this
-      // half's own score columns, already read)
-      tmem_st32(tA + 64 * half, pk);
+      // half's own score columns, already read); with dropout the dV operand
+      // is P * M (dV is scaled by 1 / (1 - p) at the end)
+      if constexpr (DROPOUT) {
+        uint32_t pd[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          pd[e] = pk[e] & (((keep_lo >> e) & 1u ? 0x0000FFFFu : 0u) | ((keep_hi >> e) & 1u ? 0xFFFF0000u : 0u));
+        tmem_st32(tA + 64 * half, pd);
+      } else {
+        tmem_st32(tA + 64 * half, pk);
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
@@ -538,12 +573,37 @@ __global__ void __launch_bounds__(512, 1)
       tmem_ld_wait(dv[0]);
       tmem_ld_wait(dv[1]);
       uint32_t dd[32];
+      if constexpr (DROPOUT) {
+        // dP'^T = dPd^T - D (extra K step).  Kept: dS = P (dPd / (1 - p) - D)
+        // = P (dP' / (1 - p) + D (1 / (1 - p) - 1)); dropped: dS = -P D.
+        // D_i of the query rows comes from their per-query row (-D in three
+        // bf16 parts, columns 9-11) in shared memory.
+        const uint8_t* ct = smem + C::CT_OFF + qs * 4096;
+        const float rp = p.drop.scale, rp1 = p.drop.scale - 1.f;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const uint32_t* src = dv[e >> 4] + 2 * (e & 15);
-        float a, b;
-        f2split(fmul2(widen2<BF16>(pk[e]), f2(__uint_as_float(src[0]), __uint_as_float(src[1]))), a, b);
-        dd[e] = pack2<BF16>(a, b);
+        for (int e = 0; e < 32; ++e) {
+          const uint32_t* src = dv[e >> 4] + 2 * (e & 15);
+          float dq[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const uint32_t qrow = (uint32_t)(64 * half + 2 * e + u);
+            const uint2 c = *reinterpret_cast<const uint2*>(ct + swz32(qrow * 32u + 16u));
+            dq[u] = -(__uint_as_float(c.x & 0xFFFF0000u) + __uint_as_float(c.y << 16) +
+                      __uint_as_float(c.y & 0xFFFF0000u));
+          }
+          const float2 pw = unpack2<BF16>(pk[e]);
+          const float a = pw.x * (((keep_lo >> e) & 1u) ? fmaf(__uint_as_float(src[0]), rp, dq[0] * rp1) : -dq[0]);
+          const float b = pw.y * (((keep_hi >> e) & 1u) ? fmaf(__uint_as_float(src[1]), rp, dq[1] * rp1) : -dq[1]);
+          dd[e] = pack2<BF16>(a, b);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const uint32_t* src = dv[e >> 4] + 2 * (e & 15);
+          float a, b;
+          f2split(fmul2(widen2<BF16>(pk[e]), f2(__uint_as_float(src[0]), __uint_as_float(src[1]))), a, b);
+          dd[e] = pack2<BF16>(a, b);
+        }
       }
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
@@ -571,7 +631,7 @@ __global__ void __launch_bounds__(512, 1)
       {
         const int which = half;  // half 0 writes dV, half 1 writes scale * dK
         uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(which ? p.dk : p.dv) + grow);
-        const float mul = which ? p.scale : 1.f;
+        const float mul = which ? p.scale : (DROPOUT ? p.drop.scale : 1.f);
         const uint32_t col = which ? C::TM_DK : C::TM_DV;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {

@@ -454,6 +454,38 @@ __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
 // 128-byte swizzle of a byte offset inside a 1024-byte-aligned block of 8
 // rows x 128 B: the 16-byte chunk index is XORed with the row index (the
 // layout TMA writes for CU_TENSOR_MAP_SWIZZLE_128B).
+// Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers:
+// as easy as 1, 2, 3", SC 2011): ten rounds, each multiplying counter words
+// 0 and 2 by the round constants and mixing the products' high halves with
+// words 1 and 3 and the round key; the key advances by the Weyl increments
+// between rounds.  Counter-based, so the dropout mask of any (head, query,
+// key) can be regenerated anywhere from its indices.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    // one 32 x 32 -> 64-bit product per multiplier gives both halves
+    uint64_t p0, p1;
+    asm("mul.wide.u32 %0, %1, %2;" : "=l"(p0) : "r"(c.x), "r"(0xD2511F53u));
+    asm("mul.wide.u32 %0, %1, %2;" : "=l"(p1) : "r"(c.z), "r"(0xCD9E8D57u));
+    c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ k0, (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ k1, (uint32_t)p0);
+  }
+  return c;
+}
+
+// Dropout parameters shared by the forward and backward kernels.  Element
+// (head bh, query i, key j) is kept when word 2 (i & 1) + (j & 1) of
+// Philox4x32-10 at counter (j >> 1, i >> 1, bh, offset), key (seed_lo,
+// seed_hi) is below `thresh` = floor((1 - p) 2^32); kept values are scaled by
+// `scale` = 1 / (1 - p).
+struct Dropout {
+  uint32_t thresh, seed_lo, seed_hi, offset;
+  float scale;
+};
+
 __device__ __forceinline__ uint32_t swz128(uint32_t off) { return off ^ (((off >> 7) & 7u) << 4); }
 // 32-byte swizzle: 16-byte chunk index (bit 4) XOR bit 7.
 __device__ __forceinline__ uint32_t swz32(uint32_t off) { return off ^ (((off >> 7) & 1u) << 4); }

@@ -195,6 +195,38 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          int deterministic, void* stream);
 
 /*
+ * Dropout on the attention probabilities (dense [B, H, S, D] batches).
+ * "Flash Attention 的算法设计原理", section "练习口述回答", lists dropout as a
+ * branch to test on its own. Because the mask must be regenerated in the
+ * backward rather than stored, it comes from a counter-based generator.
+ *
+ *   O   = (P * M / (1 - p)) V,  P = softmax(Q K^T scale [+ causal]),
+ *   LSE = that of the undropped P (as fa_fwd).
+ *
+ * M[b,h,i,j] = 1 when word 2*(i & 1) + (j & 1) of Philox4x32-10 (Salmon et
+ * al., "Parallel random numbers: as easy as 1, 2, 3", SC 2011) is below
+ * floor((1 - p) * 2^32). The counter is (j >> 1, i >> 1, b*H + h,
+ * offset mod 2^32); the key is (seed mod 2^32, seed >> 32).
+ * fa_bwd_dropout, given the same (dropout_p, seed, offset), regenerates M.
+ * It returns the gradients of sum(dO * O) for that O:
+ *   dV = (P*M/(1-p))^T dO
+ *   dS = P * (dO V^T * M/(1-p) - D),  D_i = dO_i . O_i
+ *   dQ = scale dS K,  dK = scale dS^T Q
+ *
+ * Every argument is that of fa_fwd / fa_bwd, plus dropout_p in [0, 1),
+ * seed and offset. Anything else returns FA_ERR_INVALID_ARG. dropout_p = 0
+ * is exactly fa_fwd / fa_bwd. The workspace is that of
+ * fa_bwd_workspace_size(B, H, S, D).
+ */
+fa_status fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S,
+                         int D, float scale, int causal, fa_dtype dt, float dropout_p, uint64_t seed,
+                         uint64_t offset, void* stream);
+fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int D, float scale,
+                         int causal, fa_dtype dt, int deterministic, float dropout_p, uint64_t seed,
+                         uint64_t offset, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Decode: one new query token per (sequence, query head) against a KV cache
  * ("Flash Attention 的算法设计原理", sections "训练与推理价值" and "练习口述回答":
  * at inference the new token reads the whole, growing cache, and GQA/MQA

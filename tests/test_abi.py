@@ -157,3 +157,29 @@ def test_decode_workspace_splits_and_argument_errors(lib):
     assert call(dt=5) == fa.api.FA_ERR_INVALID_ARG
     assert call(L=-1) == fa.api.FA_ERR_INVALID_ARG
     assert call(B=0) == fa.api.FA_OK                          # empty batch: nothing to do
+
+
+def test_dropout_argument_errors(lib):
+    A = 1 << 20
+    fwd = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=1, S=16, D=64, scale=0.125, causal=0, dt=0, p=0.1, seed=1,
+               off=0, stream=None)
+
+    def f(**kw):
+        a = {**fwd, **kw}
+        return fa.fa_fwd_dropout(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["S"], a["D"],
+                                 a["scale"], a["causal"], a["dt"], a["p"], a["seed"], a["off"], a["stream"])
+    assert f(p=-0.1) == fa.api.FA_ERR_INVALID_ARG
+    assert f(p=1.0) == fa.api.FA_ERR_INVALID_ARG
+    assert f(p=float("nan")) == fa.api.FA_ERR_INVALID_ARG
+    assert f(D=96) == fa.api.FA_ERR_UNSUPPORTED
+    assert f(o=A + 8) == fa.api.FA_ERR_INVALID_ARG
+    assert f(B=0) == fa.api.FA_OK
+    assert f(seed=(1 << 64) - 1, B=0) == fa.api.FA_OK          # any 64-bit seed and offset
+    need = fa.fa_bwd_workspace_size(1, 1, 64, 64)
+
+    def b(p=0.1, wsb=need, ws=A, D=64):
+        return fa.fa_bwd_dropout(*([A] * 9), 1, 1, 64, D, 0.125, 1, 0, 0, p, 7, 3, ws, wsb, None)
+    assert b(p=1.5) == fa.api.FA_ERR_INVALID_ARG
+    assert b(wsb=need - 1) == fa.api.FA_ERR_INVALID_ARG
+    assert b(ws=A + 16) == fa.api.FA_ERR_INVALID_ARG
+    assert b(D=48) == fa.api.FA_ERR_UNSUPPORTED
