@@ -61,9 +61,9 @@ def flops(w):
 # profiles/, with a digest of the kernel sources (code only) they were taken on.
 # Reported only while that code is unchanged (otherwise null: the counters are stale).
 NCU_TRAFFIC = {
-    "bwd_main": (294_589_440, "af5197c4e31d9631031a0c99a7e15f94635e740365f46ec943f2ee56522ef679",
+    "bwd_main": (290_617_088, "622027ec5545503c58134530be63b7ed0fc7cce613b1799aad5384840be6a2b6",
                  ("fa_bwd.cuh", "sm100.cuh")),
-    "fwd": (155_227_648, "bada53d807eda905390c320f5790e8c0d72f7ec6e7f34e324ed5dc10f4acab67",
+    "fwd": (151_344_000, "cc9ba07643fbca7e89ff10165cd656f83108c47abfce3c323a8694d274a5bee8",
             ("fa_fwd.cuh", "sm100.cuh")),
     # decode split kernel, B8 Hq32 Hkv8 L8192 D128 bf16, 2 splits (the merge launch is ~0.3 MB)
     "decode": (272_446_976, "c1fbc38cecaeeab210d140fe3a556f3bc1a3f4d2d1b54a558dc03779c1023e2d",
