@@ -74,6 +74,7 @@ __all__ = [
     "merge_partials",
     "philox4x32_10",
     "dropout_keep_threshold",
+    "dropout_scale",
     "dropout_keep",
     "attention_forward_dropout",
     "attention_backward_dropout",
@@ -334,19 +335,22 @@ def merge_partials(o_parts, lse_parts):
 # backward rather than stored, which needs a counter-based generator).  The
 # pages fix neither the generator nor where the mask sits, so the reading is:
 #
-# * P is the exact softmax; the output uses  Pd = P * M / (1 - p)  with
-#   M_ij in {0, 1} kept with probability 1 - p;  O = Pd V.  LSE is the
-#   statistic of the undropped softmax (dropout comes after normalisation).
-# * M_ij for head bh (= b * H + h), query i, key j is decided by one output
-#   word of Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random
+# * P is the exact softmax; the output uses  Pd = P * M * s  with M_ij in
+#   {0, 1} (kept with probability t / 2^16, t below) and s = 2^16 / t;
+#   O = Pd V.  LSE is the statistic of the undropped softmax (dropout comes
+#   after normalisation).
+# * M_ij for head bh (= b * H + h), query i, key j is decided by 16 bits of
+#   one Philox4x32-10 output (Salmon, Moraes, Dror and Shaw, "Parallel random
 #   numbers: as easy as 1, 2, 3", SC 2011) with
-#       counter = (j >> 1, i >> 1, bh, offset mod 2^32),
-#       key     = (seed mod 2^32, seed >> 32 mod 2^32),
-#   word number 2 * (i & 1) + (j & 1); the element is kept when that word is
-#   below  floor((1 - p) * 2^32).  One call covers a 2 x 2 block of (query,
-#   key), so it is as cheap to regenerate by key rows as by query rows.
+#       counter = (j >> 2, i >> 1, bh, offset mod 2^32),
+#       key     = (seed mod 2^32, seed >> 32 mod 2^32):
+#   word number 2 * (i & 1) + ((j >> 1) & 1), its low half for even j and its
+#   high half for odd j.  The element is kept when that 16-bit value is below
+#   t = floor((1 - p) * 2^16) (t >= 1), so an element is kept with
+#   probability t / 2^16 exactly, and kept values are scaled by 2^16 / t,
+#   which keeps E[O] = O exactly.  One call covers a 2 x 4 (query, key) block.
 # * Backward of L = sum(dO * O) with the same M:
-#       dV = Pd^T dO,  dPd = dO V^T,  dP = dPd * M / (1 - p),
+#       dV = Pd^T dO,  dPd = dO V^T,  dP = dPd * M * s,
 #       D_i = sum_j P_ij dP_ij  (= dO_i . O_i),  dS = P * (dP - D),
 #       dQ = scale dS K,  dK = scale dS^T Q.
 
@@ -379,33 +383,39 @@ def philox4x32_10(ctr, key):
 
 
 def dropout_keep_threshold(p: float) -> int:
-    """Integer threshold floor((1 - p) 2^32): a word below it keeps the element."""
+    """16-bit threshold t = max(1, floor((1 - p) 2^16)): a value below it keeps the element."""
     if not 0.0 <= p < 1.0:
         raise ValueError("dropout probability must be in [0, 1)")
-    return int(np.floor((1.0 - p) * 4294967296.0))
+    return max(1, int(np.floor((1.0 - p) * 65536.0)))
+
+
+def dropout_scale(p: float) -> float:
+    """Scale of the kept values, 2^16 / t (1 / the exact keep probability); 1 for p = 0."""
+    return 65536.0 / dropout_keep_threshold(p)
 
 
 def dropout_keep(bh: int, rows, cols, p: float, seed: int, offset: int) -> np.ndarray:
     """Boolean keep mask [len(rows), len(cols)] of head bh (query rows, key columns)."""
     i = np.asarray(rows, dtype=np.int64)[:, None]
     j = np.asarray(cols, dtype=np.int64)[None, :]
-    words = philox4x32_10((j >> 1, i >> 1, bh, offset & 0xFFFFFFFF), (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF))
-    sel = 2 * (i & 1) + (j & 1)
-    w = np.choose(np.broadcast_to(sel, np.broadcast_shapes(i.shape, j.shape)), words)
-    return w.astype(np.int64) < dropout_keep_threshold(p)
+    words = philox4x32_10((j >> 2, i >> 1, bh, offset & 0xFFFFFFFF), (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF))
+    sel = 2 * (i & 1) + ((j >> 1) & 1)
+    w = np.choose(np.broadcast_to(sel, np.broadcast_shapes(i.shape, j.shape)), words).astype(np.int64)
+    half = np.where((j & 1) == 1, w >> 16, w & 0xFFFF)
+    return half < dropout_keep_threshold(p)
 
 
 def _head_dropout(q, k, v, do, scale, causal, p, keep):
     s = attention_scores(q, k, scale)
     pr, m, l = _three_pass(s, _visible(q.shape[0], k.shape[0], causal))
-    pd = pr * keep / (1.0 - p)
+    pd = pr * keep * dropout_scale(p)
     o = pd @ v
     with np.errstate(divide="ignore"):
         lse = np.where(l > 0, m + np.log(l), -np.inf)
     if do is None:
         return o, lse
     dv = pd.T @ do
-    dp = (do @ v.T) * keep / (1.0 - p)
+    dp = (do @ v.T) * keep * dropout_scale(p)
     d_row = (pr * dp).sum(axis=1)
     ds = pr * (dp - d_row[:, None])
     return scale * (ds @ k), scale * (ds.T @ q), dv

@@ -49,7 +49,10 @@ def test_philox_output_statistics():
 def test_keep_rate(p):
     keep = oa.dropout_keep(5, np.arange(512), np.arange(512), p, seed=99, offset=3)
     n = keep.size
-    assert abs(keep.mean() - (1 - p)) < 5 * math.sqrt(p * (1 - p) / n)
+    q = oa.dropout_keep_threshold(p) / 65536.0  # exact keep probability, within 2^-16 of 1 - p
+    assert abs(q - (1 - p)) <= 2.0 ** -16
+    assert abs(keep.mean() - q) < 5 * math.sqrt(q * (1 - q) / n)
+    assert oa.dropout_scale(p) == 1.0 / q
 
 
 def test_mask_is_a_function_of_seed_offset_and_head():
@@ -154,7 +157,7 @@ def test_planted_mask_in_ds_fails_finite_differences():
     qq, kk, vv, dd = q[0, 0], k[0, 0], v[0, 0], do[0, 0]
     s = oa.attention_scores(qq, kk, 0.35)
     pr, _, _ = oa._three_pass(s, oa._visible(12, 12, False))
-    pd = pr * keep / (1 - p)
+    pd = pr * keep * oa.dropout_scale(p)
     dpd = dd @ vv.T
     wrong_ds = pd * (dpd - (pd * dpd).sum(axis=1, keepdims=True))
     wrong_dq = 0.35 * (wrong_ds @ kk)
