@@ -65,8 +65,8 @@ NCU_TRAFFIC = {
                  ("fa_bwd.cuh", "sm100.cuh")),
     "fwd": (151_344_000, "cc9ba07643fbca7e89ff10165cd656f83108c47abfce3c323a8694d274a5bee8",
             ("fa_fwd.cuh", "sm100.cuh")),
-    # decode split kernel, B8 Hq32 Hkv8 L8192 D128 bf16, 2 splits (the merge launch is ~0.3 MB)
-    "decode": (272_446_976, "c1fbc38cecaeeab210d140fe3a556f3bc1a3f4d2d1b54a558dc03779c1023e2d",
+    # decode split kernel, B8 Hq32 Hkv8 L8192 D128 bf16, 2 splits merged in-kernel (mean of two launches)
+    "decode": (270_329_728, "3b013eb624d2cda8538ec20903d65aea0b79831d184ee30de2bb5f28a2d52244",
                ("fa_decode.cuh", "sm100.cuh")),
 }
 

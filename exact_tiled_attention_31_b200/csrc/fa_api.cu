@@ -421,15 +421,16 @@ fa_status launch_decode_t(const fa::DecParams& p, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------- dropout
-// Keep threshold floor((1 - p) 2^32) and scale 1 / (1 - p); p in (0, 1).
+// 16-bit keep threshold t = max(1, floor((1 - p) 2^16)) and scale 2^16 / t
+// (the inverse of the exact keep probability t / 2^16); p in (0, 1).
 fa::Dropout make_dropout(float p, uint64_t seed, uint64_t offset) {
   fa::Dropout d;
-  const double keep = 1.0 - (double)p;
-  d.thresh = (uint32_t)std::min(std::floor(keep * 4294967296.0), 4294967295.0);
+  const double t = std::max(1.0, std::floor((1.0 - (double)p) * 65536.0));
+  d.thresh = (uint32_t)t;
   d.seed_lo = (uint32_t)seed;
   d.seed_hi = (uint32_t)(seed >> 32);
   d.offset = (uint32_t)offset;
-  d.scale = (float)(1.0 / keep);
+  d.scale = (float)(65536.0 / t);
   return d;
 }
 

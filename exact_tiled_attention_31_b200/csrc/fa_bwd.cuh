@@ -524,32 +524,37 @@ __global__ void __launch_bounds__(512, 1)
       }
       // dropout keep masks of the 64 query columns: bit e of keep_lo / keep_hi
       // for queries 2e and 2e + 1 of this half.  One Philox call covers query
-      // pair e x key rows (2m, 2m + 1), which sit in one lane pair: the even
-      // lane draws pairs 0-15, the odd lane 16-31, and each hands the other
-      // key row's two words across.
+      // pair e x key quad (4m .. 4m + 3), 16 bits per element, and a key quad
+      // sits in four consecutive lanes: lane 4m + c draws query pairs
+      // 8c .. 8c + 7, and each lane hands every other lane of its quad that
+      // lane's two 16-bit values (XOR shuffles over the quad).
       uint32_t keep_lo = 0xFFFFFFFFu, keep_hi = 0xFFFFFFFFu;
       if constexpr (DROPOUT) {
-        const bool odd = (lane & 1u) != 0;
-        const uint32_t th = p.drop.thresh;
-        const uint32_t keypair = (uint32_t)kv >> 1, qp0 = (uint32_t)(128 * i + 64 * half) >> 1;
+        const uint32_t c4 = lane & 3u, th = p.drop.thresh;
+        const uint32_t keyquad = (uint32_t)kv >> 2, qp0 = (uint32_t)(128 * i + 64 * half) >> 1;
         keep_lo = keep_hi = 0u;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const uint4 w = philox4x32_10(make_uint4(keypair, qp0 + k + (odd ? 16u : 0u), (uint32_t)head, p.drop.offset),
+        for (int k = 0; k < 8; ++k) {
+          const uint4 w = philox4x32_10(make_uint4(keyquad, qp0 + 8 * c4 + k, (uint32_t)head, p.drop.offset),
                                         p.drop.seed_lo, p.drop.seed_hi);
-          // word 2 * (query & 1) + (key & 1)
-          const uint32_t own0 = odd ? w.y : w.x, own1 = odd ? w.w : w.z;  // this key row
-          const uint32_t oth0 = odd ? w.x : w.y, oth1 = odd ? w.z : w.w;  // the partner key row
-          const uint32_t got0 = __shfl_xor_sync(0xffffffffu, oth0, 1), got1 = __shfl_xor_sync(0xffffffffu, oth1, 1);
-          const uint32_t a0 = odd ? got0 : own0, a1 = odd ? got1 : own1;  // query pair k
-          const uint32_t b0 = odd ? own0 : got0, b1 = odd ? own1 : got1;  // query pair 16 + k
-          keep_lo |= (a0 < th ? 1u : 0u) << k | (b0 < th ? 1u : 0u) << (16 + k);
-          keep_hi |= (a1 < th ? 1u : 0u) << k | (b1 < th ? 1u : 0u) << (16 + k);
+          // key 4m + t: word (t >> 1) for the even query, 2 + (t >> 1) for
+          // the odd one; half t & 1 of each; packed (even, odd) as 2 x 16 bits
+          auto vals_for = [&w](uint32_t t) -> uint32_t {
+            const uint32_t we = (t & 2u) ? w.y : w.x, wo = (t & 2u) ? w.w : w.z;
+            return (t & 1u) ? ((we >> 16) | (wo & 0xFFFF0000u)) : ((we & 0xFFFFu) | (wo << 16));
+          };
+#pragma unroll
+          for (uint32_t d = 0; d < 4; ++d) {
+            const uint32_t v = d == 0 ? vals_for(c4) : __shfl_xor_sync(0xffffffffu, vals_for(c4 ^ d), (int)d);
+            const uint32_t e = 8u * (c4 ^ d) + (uint32_t)k;  // query pair drawn by lane c4 ^ d
+            keep_lo |= ((v & 0xFFFFu) < th ? 1u : 0u) << e;
+            keep_hi |= ((v >> 16) < th ? 1u : 0u) << e;
+          }
         }
       }
       // P^T pairs go to columns [64*half, 64*half + 32) of A (inside this
       // half's own score columns, already read); with dropout the dV operand
-      // is P * M (dV is scaled by 1 / (1 - p) at the end)
+      // is P * M (dV is scaled by s = 1 / keep probability at the end)
       if constexpr (DROPOUT) {
         uint32_t pd[32];
 #pragma unroll
@@ -574,8 +579,8 @@ __global__ void __launch_bounds__(512, 1)
       tmem_ld_wait(dv[1]);
       uint32_t dd[32];
       if constexpr (DROPOUT) {
-        // dP'^T = dPd^T - D (extra K step).  Kept: dS = P (dPd / (1 - p) - D)
-        // = P (dP' / (1 - p) + D (1 / (1 - p) - 1)); dropped: dS = -P D.
+        // dP'^T = dPd^T - D (extra K step).  Kept: dS = P (dPd s - D)
+        // = P (dP' s + D (s - 1)); dropped: dS = -P D  (s = 1 / keep probability).
         // D_i of the query rows comes from their per-query row (-D in three
         // bf16 parts, columns 9-11) in shared memory.
         const uint8_t* ct = smem + C::CT_OFF + qs * 4096;

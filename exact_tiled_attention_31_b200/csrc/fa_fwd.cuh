@@ -42,8 +42,9 @@
 // Fully masked causal tiles are never loaded or multiplied.
 // DROPOUT instances (dense batches) zero the dropped P values before they
 // are published for the P V product, from a Philox4x32-10 mask regenerated
-// from (head, query, key) indices, and scale O by 1 / (1 - p) at the end;
-// the sums that normalise O and give LSE stay those of the undropped P.
+// from (head, query, key) indices, and scale O by 1 / (keep probability) at
+// the end; the sums that normalise O and give LSE stay those of the
+// undropped P.
 #pragma once
 
 #include "sm100.cuh"
@@ -415,25 +416,32 @@ __global__ void __launch_bounds__(768, 1)
         pk[16 + i] = exp_pair(sv[1][2 * i], sv[1][2 * i + 1], poly, fsum1, rsum1);
       }
       if constexpr (DROPOUT) {
-        // pk[e] holds keys kv0 + 2e, +1.  One Philox call covers rows
-        // (2m, 2m + 1) x key pair e, and rows 2m, 2m + 1 sit in lanes of
-        // one pair: the even lane draws pairs 0-15, the odd lane 16-31, and
-        // each hands the other row's two words across.  The sums above are
-        // of the undropped P (the softmax normaliser and LSE).
+        // pk[2q], pk[2q + 1] hold keys kv0 + 4q .. +3.  One Philox call
+        // covers rows (2m, 2m + 1) x key quad q (16 bits per element), and
+        // rows 2m, 2m + 1 sit in lanes of one pair: the even lane draws quads
+        // 0-7, the odd lane 8-15, and each hands the other row's two words
+        // across.  The sums above are of the undropped P (the softmax
+        // normaliser and LSE).
         const bool odd = (lane & 1u) != 0;
         const uint32_t th = p.drop.thresh;
-        const uint32_t rowpair = (uint32_t)row >> 1, kp0 = (uint32_t)kv0 >> 1;
+        const uint32_t rowpair = (uint32_t)row >> 1, kq0 = (uint32_t)kv0 >> 2;
+        auto keep16 = [th](uint32_t u) -> uint32_t {  // 16-bit decisions of keys 2t, 2t + 1
+          return ((u & 0xFFFFu) < th ? 0x0000FFFFu : 0u) | ((u >> 16) < th ? 0xFFFF0000u : 0u);
+        };
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const uint4 w = philox4x32_10(make_uint4(kp0 + k + (odd ? 16u : 0u), rowpair, (uint32_t)head, p.drop.offset),
+        for (int k = 0; k < 8; ++k) {
+          const uint4 w = philox4x32_10(make_uint4(kq0 + k + (odd ? 8u : 0u), rowpair, (uint32_t)head, p.drop.offset),
                                         p.drop.seed_lo, p.drop.seed_hi);
+          // word 2 * (row & 1) + ((key >> 1) & 1)
           const uint32_t own0 = odd ? w.z : w.x, own1 = odd ? w.w : w.y;  // this row
           const uint32_t oth0 = odd ? w.x : w.z, oth1 = odd ? w.y : w.w;  // the partner row
           const uint32_t got0 = __shfl_xor_sync(0xffffffffu, oth0, 1), got1 = __shfl_xor_sync(0xffffffffu, oth1, 1);
-          const uint32_t a0 = odd ? got0 : own0, a1 = odd ? got1 : own1;  // this row, pair k
-          const uint32_t b0 = odd ? own0 : got0, b1 = odd ? own1 : got1;  // this row, pair 16 + k
-          pk[k] &= (a0 < th ? 0x0000FFFFu : 0u) | (a1 < th ? 0xFFFF0000u : 0u);
-          pk[16 + k] &= (b0 < th ? 0x0000FFFFu : 0u) | (b1 < th ? 0xFFFF0000u : 0u);
+          const uint32_t a0 = odd ? got0 : own0, a1 = odd ? got1 : own1;  // this row, quad k
+          const uint32_t b0 = odd ? own0 : got0, b1 = odd ? own1 : got1;  // this row, quad 8 + k
+          pk[2 * k] &= keep16(a0);
+          pk[2 * k + 1] &= keep16(a1);
+          pk[16 + 2 * k] &= keep16(b0);
+          pk[16 + 2 * k + 1] &= keep16(b1);
         }
       }
       tmem_st32(tS + 32 * h, pk);
@@ -519,7 +527,8 @@ __global__ void __launch_bounds__(768, 1)
       const float m = t ? m_row1 : m_row0;
       const float l = sum_buf[((2 * t + 0) * 2 + 0) * 128 + r] + sum_buf[((2 * t + 1) * 2 + 0) * 128 + r];
       const float lr = sum_buf[((2 * t + 0) * 2 + 1) * 128 + r] + sum_buf[((2 * t + 1) * 2 + 1) * 128 + r];
-      // dropout: O = (P * M) V / (1 - p), P normalised by the undropped sum
+      // dropout: O = (P * M) V * s (s = 1 / keep probability), P normalised
+      // by the undropped sum
       const float inv = lr > 0.f ? (DROPOUT ? p.drop.scale : 1.f) / lr : 0.f;
       const int row = q_start + 128 * t + r;
       const bool valid = row < seq_len;

@@ -477,10 +477,11 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
 }
 
 // Dropout parameters shared by the forward and backward kernels.  Element
-// (head bh, query i, key j) is kept when word 2 (i & 1) + (j & 1) of
-// Philox4x32-10 at counter (j >> 1, i >> 1, bh, offset), key (seed_lo,
-// seed_hi) is below `thresh` = floor((1 - p) 2^32); kept values are scaled by
-// `scale` = 1 / (1 - p).
+// (head bh, query i, key j) is kept when half (j & 1) (low for even j) of
+// word 2 (i & 1) + ((j >> 1) & 1) of Philox4x32-10 at counter (j >> 2,
+// i >> 1, bh, offset), key (seed_lo, seed_hi), is below `thresh` =
+// max(1, floor((1 - p) 2^16)); kept values are scaled by `scale` =
+// 2^16 / thresh, the inverse of the exact keep probability.
 struct Dropout {
   uint32_t thresh, seed_lo, seed_hi, offset;
   float scale;

@@ -200,17 +200,21 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
  * branch to test on its own. Because the mask must be regenerated in the
  * backward rather than stored, it comes from a counter-based generator.
  *
- *   O   = (P * M / (1 - p)) V,  P = softmax(Q K^T scale [+ causal]),
+ *   O   = (P * M * s) V,  P = softmax(Q K^T scale [+ causal]),
  *   LSE = that of the undropped P (as fa_fwd).
  *
- * M[b,h,i,j] = 1 when word 2*(i & 1) + (j & 1) of Philox4x32-10 (Salmon et
- * al., "Parallel random numbers: as easy as 1, 2, 3", SC 2011) is below
- * floor((1 - p) * 2^32). The counter is (j >> 1, i >> 1, b*H + h,
- * offset mod 2^32); the key is (seed mod 2^32, seed >> 32).
+ * The mask M[b,h,i,j] comes from Philox4x32-10 (Salmon et al., "Parallel
+ * random numbers: as easy as 1, 2, 3", SC 2011):
+ *   - counter (j >> 2, i >> 1, b*H + h, offset mod 2^32);
+ *   - key (seed mod 2^32, seed >> 32);
+ *   - word 2*(i & 1) + ((j >> 1) & 1), low half for even j, high half for odd j.
+ * M = 1 when that 16-bit value is below t = max(1, floor((1 - p) * 2^16)).
+ * An element is therefore kept with probability t / 2^16, and s = 2^16 / t
+ * keeps E[O] exact.
  * fa_bwd_dropout, given the same (dropout_p, seed, offset), regenerates M.
  * It returns the gradients of sum(dO * O) for that O:
- *   dV = (P*M/(1-p))^T dO
- *   dS = P * (dO V^T * M/(1-p) - D),  D_i = dO_i . O_i
+ *   dV = (P*M*s)^T dO
+ *   dS = P * (dO V^T * M*s - D),  D_i = dO_i . O_i
  *   dQ = scale dS K,  dK = scale dS^T Q
  *
  * Every argument is that of fa_fwd / fa_bwd, plus dropout_p in [0, 1),
