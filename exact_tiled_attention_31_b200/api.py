@@ -264,14 +264,19 @@ def forward_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool, scale: fl
 
 
 def backward(q, k, v, o, do, lse, causal: bool, scale: float | None = None, deterministic: bool = False,
-             workspace=None, stream=None, dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
+             workspace=None, stream=None, dropout_p: float = 0.0, seed: int = 0, offset: int = 0, out=None):
     """dQ, dK, dV of [B, H, S, D] inputs given the forward's O and LSE (and
-    the forward's dropout_p, seed and offset, if it dropped)."""
+    the forward's dropout_p, seed and offset, if it dropped).  ``out`` may
+    give the three output tensors to fill."""
     import torch
     B, H, S, D = q.shape
     _check((q, k, v, o, do), q.shape)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if out is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        dq, dk, dv = out
+        _check((q, dq, dk, dv), q.shape)
     nbytes = fa_bwd_workspace_size(B, H, S, D)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(max(nbytes, 1), device=q.device, dtype=torch.uint8)
