@@ -4,7 +4,7 @@
 compiles ``csrc/fa_api.cu`` (which includes the kernels) for
 ``arch=compute_100a, code=sm_100a`` and links the CUDA runtime statically, so
 the library loads on a machine without a GPU (for the export checks) and
-needs no JIT cache on the GPU machine.
+needs no JIT cache on the machine that runs it.
 """
 from __future__ import annotations
 
