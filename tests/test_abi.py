@@ -183,3 +183,16 @@ def test_dropout_argument_errors(lib):
     assert b(wsb=need - 1) == fa.api.FA_ERR_INVALID_ARG
     assert b(ws=A + 16) == fa.api.FA_ERR_INVALID_ARG
     assert b(D=48) == fa.api.FA_ERR_UNSUPPORTED
+
+
+def test_decode_split_rule():
+    """The library's split count: the fewest splits giving about 0.8 x 148
+    CTAs (one B200 wave), at least 256 keys each, at most 64 (148 SMs is the
+    count the library assumes when no device answers)."""
+    import math
+    for B, Hkv, L in [(8, 8, 8192), (1, 8, 32768), (32, 8, 2048), (8, 32, 4096), (16, 1, 8192), (64, 8, 1024),
+                      (1, 1, 1 << 20), (2, 4, 300)]:
+        target = (8 * 148 + 9) // 10
+        nmax = max(1, min(64, ((L + 31) // 32) // 8))
+        expect = max(1, min(nmax, math.ceil(target / (B * Hkv))))
+        assert fa.fa_decode_num_splits(B, Hkv, L) == expect, (B, Hkv, L)
