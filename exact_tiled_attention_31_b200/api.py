@@ -2,14 +2,16 @@
 
 Two layers:
 
-* ``fa_fwd``, ``fa_fwd_varlen``, ``fa_bwd_workspace_size``, ``fa_bwd``,
-  ``fa_status_string``, ``fa_check_device_error``, ``fa_launch_count``: the C
-  entry points under the same names, taking raw device pointers (ints) and
-  sizes, returning the ``fa_status`` code.
-* ``forward``, ``forward_varlen``, ``backward``: tensor conveniences that
-  check shapes/dtypes, allocate outputs and workspace with torch (device
-  memory and the current stream are all torch provides) and raise
-  ``FAError`` on a non-zero status.
+* ``fa_*`` (every name in ``EXPORTS``: forward, packed forward, the
+  backward and its three launches, the packed and allocation-free
+  backwards, dropout forward/backward, decode, status and error helpers):
+  the C entry points under the same names, taking raw device pointers (ints)
+  and sizes, returning the ``fa_status`` code (or a size).
+* ``forward``, ``forward_varlen``, ``backward``, ``backward_varlen``,
+  ``backward_noalloc``, ``decode``: tensor conveniences that check
+  shapes/dtypes, allocate outputs and workspace with torch unless given
+  (device memory and streams are all torch provides) and raise ``FAError``
+  on a non-zero status.
 
 Every step of the attention itself runs in the library's CUDA kernels; there
 is no fallback.  If ``libfa.so`` is missing, every call raises.
