@@ -46,6 +46,19 @@ def test_decode_matches_oracle(cuda_device, Hq, Hkv, D, dtype, n_splits):
     check_lse(lse, rl, "decode LSE")
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,D,dtype,n_splits", [
+    (4, 16, 4, 64, "bf16", 2),      # D = 64 splits merged in-kernel (2-CTA clusters, 32 CTAs)
+    (3, 8, 8, 64, "fp16", 4),       # D = 64, 4-CTA clusters
+    (40, 8, 4, 128, "bf16", 4),     # 4 splits over 160 CTAs (more than one wave): merge kernel
+])
+def test_decode_merge_paths(cuda_device, B, Hq, Hkv, D, dtype, n_splits):
+    t = inputs.make_decode(B, Hq, Hkv, 600, D, dtype, seed=B + D)
+    o, lse = _run(t, cuda_device, n_splits)
+    ro, rl = _ref(t, 1.0 / math.sqrt(D))
+    check_o(o, ro, f"decode merge path B{B} Hq{Hq} Hkv{Hkv} D{D} splits {n_splits}")
+    check_lse(lse, rl, "decode merge path LSE")
+
+
 def test_decode_ragged_lengths_and_edges(cuda_device):
     """Lengths at and around the 32-key tile, a single key, the full cache,
     a length past the cache (clamped to L_max) and an empty sequence
