@@ -69,6 +69,10 @@ def test_backward_mask_is_the_oracle_mask(cuda_device, causal):
     (1, 3, 517, 128, "fp16", False, 0.3),
     (1, 2, 1024, 128, "bf16", True, 0.5),
     (2, 2, 129, 64, "fp16", False, 0.2),
+    # the remaining kernel instances (D x dtype x causal)
+    (1, 2, 257, 64, "bf16", False, 0.15),
+    (1, 2, 384, 64, "fp16", True, 0.25),
+    (1, 2, 200, 128, "fp16", True, 0.4),
 ])
 def test_dropout_forward_backward_match_oracle(cuda_device, B, H, S, D, dtype, causal, p):
     q, k, v, do = _rand(B, H, S, D, dtype, seed=S + D)
