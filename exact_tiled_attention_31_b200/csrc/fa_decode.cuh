@@ -237,8 +237,9 @@ __global__ void __launch_bounds__(128, 1)
     const int t = warp + C::WARPS * i, st = i % C::STAGES;
     if (full_tile(i)) {
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[warp][st], (i / C::STAGES) & 1, DEC_SITE_KV));
-      if (!ok) {  // error recorded: let the warp's copies in flight land (bounded), then stop
-        for (int j = i + 1; j < min(i + C::STAGES, my_tiles); ++j)
+      if (!ok) {  // error recorded: let the warp's copies in flight, this tile's included, land
+                  // (bounded waits again), then stop
+        for (int j = i; j < min(i + C::STAGES, my_tiles); ++j)
           if (full_tile(j)) mbar_wait(&bars[warp][j % C::STAGES], (j / C::STAGES) & 1, DEC_SITE_DRAIN);
         break;
       }
