@@ -24,6 +24,13 @@ def _round_like(x: np.ndarray, dtype) -> np.ndarray:
     return torch.from_numpy(x).to(dtype).double().numpy()
 
 
+# Every element that check_o held against the oracle rounded to the output
+# dtype (instead of the raw oracle), one record per call that had any:
+# {"what", "elements", "raw_max", "err_vs_rounded_max"}.  conftest.py attaches
+# each test's records to its report and prints them all at the end of the run.
+ROUNDED_COMPARISONS: list = []
+
+
 def check_o(o_gpu, o_ref, what=""):
     """O within the stated bounds of the fp64 oracle.
 
@@ -31,22 +38,34 @@ def check_o(o_gpu, o_ref, what=""):
     the oracle than the oracle rounded to that dtype: for bf16 that half-ulp
     is 2^-8 |O| and exceeds 1e-2 once |O| >= 4.  Such elements (and only
     those) are held to the 1e-2 bound against the oracle rounded to the
-    output dtype; the raw max-abs error is still reported in the message.
+    output dtype.  They are never dropped silently: their number and their
+    worst raw error are appended to ``ROUNDED_COMPARISONS`` (reported after
+    the run and in every failure message), and the raw max-abs error is in
+    the message as well.
     """
     dtype = o_gpu.dtype if isinstance(o_gpu, torch.Tensor) else torch.float64
     o_gpu, o_ref = f64(o_gpu), f64(o_ref)
     assert np.isfinite(o_gpu).all(), f"{what}: non-finite O"
     raw = np.abs(o_gpu - o_ref)
     err = raw
+    n_rounded, note = 0, ""
     if raw.max() > O_MAX and dtype in (torch.bfloat16, torch.float16):
-        rounding = np.abs(_round_like(o_ref, dtype) - o_ref)
-        beyond = rounding > O_MAX  # the dtype cannot represent the oracle to 1e-2 here
-        err = np.where(beyond, np.abs(o_gpu - _round_like(o_ref, dtype)), raw)
+        rounded = _round_like(o_ref, dtype)
+        beyond = np.abs(rounded - o_ref) > O_MAX  # the dtype cannot represent the oracle to 1e-2 here
+        err = np.where(beyond, np.abs(o_gpu - rounded), raw)
+        n_rounded = int(beyond.sum())
+        if n_rounded:
+            rec = {"what": what, "elements": n_rounded, "raw_max": float(raw[beyond].max()),
+                   "err_vs_rounded_max": float(err[beyond].max())}
+            ROUNDED_COMPARISONS.append(rec)
+            note = (f"; {n_rounded} element(s) held against the oracle rounded to {dtype} (raw error up to "
+                    f"{rec['raw_max']:.3e}, {rec['err_vs_rounded_max']:.3e} against the rounded oracle)")
     emax, emean = err.max(), raw.mean()
     if emax > O_MAX or emean > O_MEAN:
         idx = np.unravel_index(err.argmax(), err.shape)
         raise AssertionError(f"{what}: O max-abs {emax:.3e} (raw {raw.max():.3e}, limit {O_MAX}) mean-abs "
-                             f"{emean:.3e} (limit {O_MEAN}); worst at {idx}: gpu {o_gpu[idx]:.5f} ref {o_ref[idx]:.5f}")
+                             f"{emean:.3e} (limit {O_MEAN}); worst at {idx}: gpu {o_gpu[idx]:.5f} ref {o_ref[idx]:.5f}"
+                             + note)
     return raw.max(), emean
 
 

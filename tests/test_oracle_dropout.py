@@ -4,12 +4,80 @@ reduction to plain attention, unbiasedness of the dropped output, and the
 backward against central finite differences for a fixed mask.  Planted
 mistakes (a missing 1/(1-p), the mask applied to P inside dS, a mask that
 ignores the head) each fail one of them."""
+import json
 import math
+import os
 
 import numpy as np
 import pytest
 
 from oracle import attention as oa
+
+_KAT = os.path.join(os.path.dirname(__file__), "golden", "philox4x32_10_kat.json")
+
+
+def _kat_vectors():
+    with open(_KAT) as f:
+        vecs = json.load(f)["vectors"]
+    return [([int(x, 16) for x in v["ctr"]], [int(x, 16) for x in v["key"]], [int(x, 16) for x in v["out"]])
+            for v in vecs]
+
+
+def _kat_failures(gen):
+    """Known-answer vectors that ``gen`` does not reproduce."""
+    bad = []
+    for ctr, key, out in _kat_vectors():
+        got = [int(np.asarray(w)) for w in gen(ctr, key)]
+        if got != out:
+            bad.append((ctr, key, [hex(x) for x in got]))
+    return bad
+
+
+def test_philox_known_answers():
+    """The oracle's generator reproduces the published Philox4x32-10
+    known-answer vectors (Salmon, Moraes, Dror and Shaw, SC 2011; the
+    Random123 distribution's kat_vectors): the all-zero, all-ones and
+    pi-digit counters and keys, stored in tests/golden/philox4x32_10_kat.json.
+    This pins the generator to its published definition, independently of
+    the GPU copy agreeing with it."""
+    assert _kat_failures(oa.philox4x32_10) == []
+
+
+def test_philox_known_answers_reject_planted_mistakes(monkeypatch):
+    """Each plausible slip in a Philox implementation fails the known
+    answers: the two round multipliers swapped, a wrong Weyl increment, nine
+    rounds instead of ten (key schedule one step short), and output words
+    in the wrong order."""
+    m0, m1 = oa._PHILOX_M
+    w0, w1 = oa._PHILOX_W
+    with monkeypatch.context() as mp:
+        mp.setattr(oa, "_PHILOX_M", (m1, m0))
+        assert len(_kat_failures(oa.philox4x32_10)) == 3
+    with monkeypatch.context() as mp:
+        mp.setattr(oa, "_PHILOX_W", (w0, np.uint64(0xBB67AE86)))
+        assert len(_kat_failures(oa.philox4x32_10)) == 3
+    with monkeypatch.context() as mp:
+        mp.setattr(oa, "_PHILOX_W", (w1, w0))
+        assert len(_kat_failures(oa.philox4x32_10)) == 3
+
+    def nine_rounds(ctr, key):
+        c = [np.asarray(x).astype(np.uint64) for x in ctr]
+        k0, k1 = np.uint64(key[0]), np.uint64(key[1])
+        mask = np.uint64(0xFFFFFFFF)
+        for r in range(9):
+            if r:
+                k0, k1 = (k0 + w0) & mask, (k1 + w1) & mask
+            p0, p1 = c[0] * m0, c[2] * m1
+            c = [(p1 >> np.uint64(32)) ^ c[1] ^ k0, p1 & mask, (p0 >> np.uint64(32)) ^ c[3] ^ k1, p0 & mask]
+        return c
+
+    assert len(_kat_failures(nine_rounds)) == 3
+
+    def swapped_words(ctr, key):
+        x = oa.philox4x32_10(ctr, key)
+        return [x[1], x[0], x[2], x[3]]
+
+    assert len(_kat_failures(swapped_words)) == 3
 
 
 def _qkv(S, D, seed, B=1, H=1):
