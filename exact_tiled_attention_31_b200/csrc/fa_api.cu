@@ -11,6 +11,7 @@
 #include <cstring>
 #include <initializer_list>
 #include <mutex>
+#include <utility>
 
 #include "../../include/fa.h"
 #include "fa_bwd.cuh"
@@ -324,20 +325,52 @@ __global__ void __launch_bounds__(32) selftest_timeout_kernel() {
 // device address is looked up once per device below.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch on the current device, looked up on
-// the first call per device (with that device current) and cached.
+// Process-unique id of the calling thread's current CUDA context
+// (cuCtxGetId), or 0 when the driver does not offer it.  Ids are never
+// reused within a process, unlike context handles after a reset.
+unsigned long long current_context_id() {
+  using GetCurrentFn = CUresult (*)(CUcontext*);
+  using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static const std::pair<GetCurrentFn, GetIdFn> fns = []() -> std::pair<GetCurrentFn, GetIdFn> {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+        qa != cudaDriverEntryPointSuccess || cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+        qb != cudaDriverEntryPointSuccess)
+      return {nullptr, nullptr};
+    return {reinterpret_cast<GetCurrentFn>(a), reinterpret_cast<GetIdFn>(b)};
+  }();
+  if (!fns.first || !fns.second) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (fns.first(&ctx) != CUDA_SUCCESS || !ctx || fns.second(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch in the current device's context.  It
+// is looked up (cudaGetSymbolAddress, with the device current; no
+// allocation) on the first call in a context and cached together with that
+// context's id, so a later call from another context, or after the device
+// was reset, looks it up again instead of reusing an address of a context
+// that no longer exists.  Without context ids it is looked up on every call.
 void* noalloc_scratch() {
+  struct Entry {
+    unsigned long long ctx;
+    void* addr;
+  };
   static std::mutex mu;
-  static void* addr[64] = {};
+  static Entry cache[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (cudaSetDevice(dev) != cudaSuccess) return nullptr;  // makes the device's primary context current
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = p;
-  }
-  return addr[dev];
+  if (ctx != 0 && cache[dev].ctx == ctx && cache[dev].addr) return cache[dev].addr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+  cache[dev] = Entry{ctx, p};
+  return p;
 }
 
 // ---------------------------------------------------------------- decode

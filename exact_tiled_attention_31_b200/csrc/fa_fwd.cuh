@@ -86,15 +86,6 @@ struct FwdCfg {
   static constexpr int THREADS = 768;
 };
 
-// Row-max growth (log2 units) tolerated before O and l are rescaled.  Zero
-// keeps the exact running max, so the dominant P of every row is exactly 1
-// and only the smaller weights carry 16-bit rounding into P V.
-constexpr float kRescaleLog2 = 0.f;
-
-// One pair in kPolyEvery of a fully visible score tile is exponentiated on
-// the FMA pipe (exp2_poly2) instead of the special-function unit; 0 = never.
-constexpr int kPolyEvery = 0;
-
 // wait-site ids reported through the error word
 enum : uint32_t {
   FWD_SITE_PROD = 0x100, FWD_SITE_Q = 0x101, FWD_SITE_KV = 0x102, FWD_SITE_P = 0x103, FWD_SITE_S = 0x104,
@@ -348,8 +339,7 @@ __global__ void __launch_bounds__(768, 1)
       const int kv0 = 128 * j + 64 * h;
       int limit = min(64, seq_len - kv0);
       if constexpr (CAUSAL) limit = min(limit, row - kv0 + 1);
-      const bool full = limit >= 64;
-      if (!full) {
+      if (limit < 64) {
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -376,29 +366,23 @@ __global__ void __launch_bounds__(768, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&mx_full[t], j & 1, FWD_SITE_MX));
       if (!ok) break;
       const float mx = fmaxf(pm, *other_max);
-      // Rescale only when the row max actually grew (by more than
-      // kRescaleLog2): every P is then <= 2^kRescaleLog2, and with
-      // kRescaleLog2 = 0 the largest P of the row is exactly 1.  The
-      // correction warpgroup makes the same decision from the same values.
-      const float m_max = fmaxf(m, mx * sl2);
-      const bool rescale = m_max > m + kRescaleLog2;  // false while the row has no visible key
-      const float m_new = rescale ? m_max : m;
-      const float alpha = rescale ? ex2(m - m_new) : 1.f;  // ex2(-inf) = 0 on the first tile
+      // Exact running max: rescale whenever the row max grows, so the
+      // largest P of the row is exactly 1 and only the smaller weights carry
+      // 16-bit rounding into P V.  The correction warpgroup makes the same
+      // decision from the same values.
+      const float m_new = fmaxf(m, mx * sl2);
+      const float alpha = m_new > m ? ex2(m - m_new) : 1.f;  // ex2(-inf) = 0 on the first tile
       const float neg = (m_new == -INFINITY) ? 0.f : -m_new;
       const uint64_t scale2 = f2(sl2, sl2), neg2 = f2(neg, neg);
       // fsum: fp32 sum of P (for LSE); rsum: sum of P as rounded to 16 bits
       // (the weights the P V product uses, for normalising O).
       uint64_t fsum0 = f2(0.f, 0.f), fsum1 = f2(0.f, 0.f), rsum0 = f2(0.f, 0.f), rsum1 = f2(0.f, 0.f);
-      auto exp_pair = [&](uint32_t x, uint32_t y, bool poly, uint64_t& fs, uint64_t& rs) -> uint32_t {
+      auto exp_pair = [&](uint32_t x, uint32_t y, uint64_t& fs, uint64_t& rs) -> uint32_t {
         const uint64_t arg = ffma2(f2(__uint_as_float(x), __uint_as_float(y)), scale2, neg2);
         float a, bb;
-        if (poly) {
-          f2split(exp2_poly2(arg), a, bb);
-        } else {
-          f2split(arg, a, bb);
-          a = ex2(a);
-          bb = ex2(bb);
-        }
+        f2split(arg, a, bb);
+        a = ex2(a);
+        bb = ex2(bb);
         fs = fadd2(fs, f2(a, bb));
         const uint32_t pk = pack2<BF16>(a, bb);
         rs = fadd2(rs, widen2<BF16>(pk));
@@ -410,10 +394,8 @@ __global__ void __launch_bounds__(768, 1)
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        constexpr int every = kPolyEvery > 0 ? kPolyEvery : 1;
-        const bool poly = kPolyEvery > 0 && full && (i % every) == every - 1;
-        pk[i] = exp_pair(sv[0][2 * i], sv[0][2 * i + 1], poly, fsum0, rsum0);
-        pk[16 + i] = exp_pair(sv[1][2 * i], sv[1][2 * i + 1], poly, fsum1, rsum1);
+        pk[i] = exp_pair(sv[0][2 * i], sv[0][2 * i + 1], fsum0, rsum0);
+        pk[16 + i] = exp_pair(sv[1][2 * i], sv[1][2 * i + 1], fsum1, rsum1);
       }
       if constexpr (DROPOUT) {
         // pk[2q], pk[2q + 1] hold keys kv0 + 4q .. +3.  One Philox call
@@ -481,10 +463,8 @@ __global__ void __launch_bounds__(768, 1)
         if (!ok) break;
         const float mx = fmaxf(pmax_buf[(2 * t) * 128 + r], pmax_buf[(2 * t + 1) * 128 + r]);
         const float m = t ? m_row1 : m_row0;
-        const float m_max = fmaxf(m, mx * sl2);
-        const bool rescale = m_max > m + kRescaleLog2;
-        const float m_new = rescale ? m_max : m;
-        const float alpha = rescale ? ex2(m - m_new) : 1.f;
+        const float m_new = fmaxf(m, mx * sl2);
+        const float alpha = m_new > m ? ex2(m - m_new) : 1.f;
         if (t) m_row1 = m_new; else m_row0 = m_new;
         // O_t is written fresh by the first P V product; later, if any factor
         // differs from 1, wait for the previous P V product of tile t, then

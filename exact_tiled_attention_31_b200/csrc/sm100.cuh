@@ -362,32 +362,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of x <= 8 on the FMA and integer pipes (no special-function
-// unit).  Cody-Waite style range reduction: x = j + f with j the nearest
-// integer (adding and subtracting 1.5 * 2^23 rounds to an integer and leaves
-// j in the low mantissa bits of the sum) and f in [-1/2, 1/2]; 2^f by the
-// cubic p(f) = 1 + c1 f + c2 f^2 + c3 f^3 fitted in csrc/fit_exp2_poly.py
-// (max relative error 1.0e-4, p(0) = 1 exactly); 2^j is added to the
-// exponent field.  x is clamped at -125 so the result stays a normal float
-// (2^-125 stands for anything smaller).
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
-  constexpr float c1 = 0.6932829022407532f, c2 = 0.24221095442771912f, c3 = 0.05500892922282219f;
-  float xa, xb;
-  f2split(x2, xa, xb);
-  x2 = f2(fmaxf(xa, -125.f), fmaxf(xb, -125.f));
-  const uint64_t t2 = fadd2(x2, f2(kRound, kRound));
-  const uint64_t fr = fadd2(x2, fadd2(t2, f2(-kRound, -kRound)) ^ 0x8000000080000000ull);  // x - (t - kRound)
-  uint64_t p2 = ffma2(f2(c3, c3), fr, f2(c2, c2));
-  p2 = ffma2(p2, fr, f2(c1, c1));
-  p2 = ffma2(p2, fr, f2(1.f, 1.f));
-  float pa, pb, ta, tb;
-  f2split(p2, pa, pb);
-  f2split(t2, ta, tb);
-  return f2(__int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23)),
-            __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23)));
-}
-
 // Two fp32 values rounded to nearest into one packed 16-bit pair: `lo` in
 // bits 0-15 (the lower column / element index), `hi` in bits 16-31.
 template <bool BF16>
@@ -451,9 +425,6 @@ __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// 128-byte swizzle of a byte offset inside a 1024-byte-aligned block of 8
-// rows x 128 B: the 16-byte chunk index is XORed with the row index (the
-// layout TMA writes for CU_TENSOR_MAP_SWIZZLE_128B).
 // Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers:
 // as easy as 1, 2, 3", SC 2011): ten rounds, each multiplying counter words
 // 0 and 2 by the round constants and mixing the products' high halves with
@@ -487,6 +458,9 @@ struct Dropout {
   float scale;
 };
 
+// 128-byte swizzle of a byte offset inside a 1024-byte-aligned block of 8
+// rows x 128 B: the 16-byte chunk index is XORed with the row index (the
+// layout TMA writes for CU_TENSOR_MAP_SWIZZLE_128B).
 __device__ __forceinline__ uint32_t swz128(uint32_t off) { return off ^ (((off >> 7) & 7u) << 4); }
 // 32-byte swizzle: 16-byte chunk index (bit 4) XOR bit 7.
 __device__ __forceinline__ uint32_t swz32(uint32_t off) { return off ^ (((off >> 7) & 1u) << 4); }

@@ -95,6 +95,10 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
  * D_i = dO_i . O_i, as bf16 parts, rows padded to multiples of 128), and the
  * ordering counters of deterministic mode, each 256-byte aligned.
  * Returns 0 for unsupported sizes.
+ * This is the first half of the two-phase call of the operator in
+ * "ops-transformer里的FlashAttention", "ops-transformer里的完整算子": a size
+ * query for the workspace (there aclnnFlashAttentionGetWorkspaceSize), then
+ * the computation given a caller-allocated workspace of that size.
  */
 size_t fa_bwd_workspace_size(int B, int H, int S, int D);
 
@@ -105,7 +109,8 @@ size_t fa_bwd_workspace_size(int B, int H, int S, int D);
  * fa_bwd_workspace_size(B, H, S, D) bytes, 256-byte aligned; its contents on
  * entry do not matter and are overwritten.
  * deterministic = 0: dQ partial sums from different key tiles are added with
- *   fp32 atomics, so dq may differ in the last bits from run to run.
+ *   fp32 reductions (TMA bulk reduce-adds) in whatever order the key tiles
+ *   reach them, so dq may differ in the last bits from run to run.
  * deterministic = 1: the key tiles of one query tile add their dQ partials in
  *   increasing key-tile order, so repeated calls with the same inputs, sizes
  *   and GPU give bit-identical dq (the `deterministic` option of the
@@ -136,6 +141,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * are a branch to test on their own) and "核心机制" (recompute P from the
  * saved statistics).  nseq, H, total or max_seqlen equal to 0 is a no-op.
  */
+/* Workspace size query of fa_bwd_varlen: the same two-phase call as
+ * fa_bwd_workspace_size ("ops-transformer里的完整算子"); 0 for unsupported sizes. */
 size_t fa_bwd_varlen_workspace_size(int nseq, int max_seqlen, int total, int H, int D);
 fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dO,
                         const float* lse, void* dq, void* dk, void* dv,
@@ -144,7 +151,8 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
                         int deterministic, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * The three launches fa_bwd makes, exposed for callers that want to place
+ * The three launches fa_bwd makes (the pages describe the backward as one
+ * operator; the split only exposes its phases), exposed for callers that want to place
  * or time them separately (same arguments, same rules, same workspace; they
  * must run in this order on one stream):
  *   fa_bwd_preprocess  D_i = dO_i . O_i and LSE into the workspace (as
@@ -178,9 +186,11 @@ fa_status fa_bwd_finish(void* dq, int B, int H, int S, int D, float scale, fa_dt
  * process exits.  The caller still provides every input and output.
  *   - Sizes with fa_bwd_workspace_size(B, H, S, D) > FA_BWD_NOALLOC_SCRATCH_BYTES
  *     are refused with FA_ERR_UNSUPPORTED before anything is launched.
- *   - The first call on each device looks up that array's device address
- *     (with the device current) and caches it; make that first call before
- *     any stream capture.
+ *   - The first call in each device context looks up that array's device
+ *     address (with the device current) and caches it with the context's
+ *     process-unique id; make that first call before any stream capture.
+ *     A call from another context, or after cudaDeviceReset, looks the
+ *     address up again rather than reuse one of a context that is gone.
  *   - Every call on a device shares the one array, which keeps the previous
  *     call's contents; each call clears what must start at zero itself.
  *     Calls whose kernels overlap on the GPU (different streams without
@@ -262,19 +272,24 @@ fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void
  * otherwise); B, Hkv <= 65535; q, k_cache, v_cache, o, lse 16-byte aligned.
  * B = 0 or Hq = 0 is a no-op.  Two kernel launches on `stream`.
  */
+/* The library's split count for fa_decode at these sizes (the key ranges of
+ * "训练与推理价值"'s decode over a long cache; the pages give no rule, this one
+ * is measured on B200). */
 int fa_decode_num_splits(int B, int Hkv, int L_max);
 size_t fa_decode_workspace_size(int B, int Hq, int n_splits, int D);
 fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, const int* seq_lens, void* o,
                     float* lse, int B, int Hq, int Hkv, int L_max, int D, float scale, fa_dtype dt,
                     int n_splits, void* workspace, size_t workspace_bytes, void* stream);
 
-/* A static, human-readable name for a status code. */
+/* A static, human-readable name for a status code.  No page defines status
+ * codes; they are this library's error reporting. */
 const char* fa_status_string(fa_status s);
 
 /*
  * Synchronises `stream`, then reads and clears the calling device's error
  * word.  Returns FA_OK, FA_ERR_TIMEOUT (a kernel gave up waiting) or
- * FA_ERR_CUDA (the synchronisation itself failed).
+ * FA_ERR_CUDA (the synchronisation itself failed).  No page defines this
+ * call; it is the host side of the library's bounded-wait error handling.
  */
 fa_status fa_check_device_error(void* stream);
 
@@ -288,7 +303,8 @@ fa_status fa_check_device_error(void* stream);
  */
 fa_status fa_selftest_timeout(void* stream);
 
-/* Number of kernel launches issued by this process through the library so far. */
+/* Number of kernel launches issued by this process through the library so
+ * far (for checking that the native path ran).  No page defines this call. */
 uint64_t fa_launch_count(void);
 
 #ifdef __cplusplus
