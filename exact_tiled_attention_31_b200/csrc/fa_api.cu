@@ -167,7 +167,7 @@ fa_status run_fwd(const void* q, const void* k, const void* v, void* o, float* l
 
 // ---------------------------------------------------------------- backward
 struct WsLayout {
-  size_t dq_acc, cols, sem, total;
+  size_t dq_acc, cols, sem, ticket, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -180,7 +180,8 @@ WsLayout ws_layout(long long heads, long long nseq, long long S, long long rows,
   w.dq_acc = 0;
   w.cols = up256((size_t)heads * rows * D * 4);
   w.sem = w.cols + up256((size_t)heads * nseq * S_pad * 32);
-  w.total = w.sem + up256((size_t)heads * nseq * n_q * 4);
+  w.ticket = w.sem + up256((size_t)heads * nseq * n_q * 4);
+  w.total = w.ticket + 256;
   return w;
 }
 
@@ -193,6 +194,7 @@ fa::BwdParams bwd_params(int heads, int nseq, int S, int rows, const int* cu, in
   p.dq_acc = reinterpret_cast<float*>(ws + w.dq_acc);
   p.cols = reinterpret_cast<uint16_t*>(ws + w.cols);
   p.sem = reinterpret_cast<uint32_t*>(ws + w.sem);
+  p.ticket = reinterpret_cast<uint32_t*>(ws + w.ticket);
   p.cu_seqlens = cu;
   p.heads = heads;
   p.S = S;
@@ -200,6 +202,9 @@ fa::BwdParams bwd_params(int heads, int nseq, int S, int rows, const int* cu, in
   p.nseq = nseq;
   p.n_q = (S + 127) / 128;
   p.S_pad = p.n_q * 128;
+  const long long groups = ((long long)heads * nseq + fa::kBwdGroup - 1) / fa::kBwdGroup;
+  const long long units = groups * fa::kBwdGroup * p.n_q;
+  p.units = units > 0x7fffffffLL ? -1 : (int)units;  // -1: too many for one launch
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.deterministic = deterministic;
@@ -225,11 +230,11 @@ fa_status launch_bwd_main_t(const CUtensorMap& mq, const CUtensorMap& mk, const 
                             const CUtensorMap& mdo, const CUtensorMap& mdq, const CUtensorMap& mcols,
                             const fa::BwdParams& p, cudaStream_t st) {
   using C = fa::BwdCfg<D>;
-  // groups of kBwdGroup (sequence, head) slices, n_q key tiles each
-  const long long units = (long long)p.nseq * p.heads;
-  const long long groups = (units + fa::kBwdGroup - 1) / fa::kBwdGroup;
-  const long long grid = groups * fa::kBwdGroup * p.n_q;
-  if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  // persistent grid: at most one CTA per SM, each claiming units from the
+  // workspace counter that bwd_pre zeroed
+  if (p.units < 0) return FA_ERR_UNSUPPORTED;
+  if (p.units == 0) return FA_OK;
+  const int grid = std::min(p.units, sm_count());
   if (set_smem<fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN, DROPOUT>>(C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
   fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN, DROPOUT><<<(unsigned)grid, 512, C::SMEM, st>>>(mq, mk, mv, mdo, mdq,
                                                                                            mcols, p);

@@ -16,40 +16,54 @@
 //             16-column bf16 row holding -LSE_i*log2(e) and -D_i, each split
 //             into three bf16 parts (128-row padded); zero the fp32 dQ
 //             accumulator and the ordering counters.
-//   bwd_main  one CTA per 128-row key/value tile j of one head (and, for a
-//             packed batch, one sequence; 512 threads):
-//               warp 0     TMA producer: K_j, V_j once; then Q_i (+ the
-//                          per-query rows of tile i) into a 2-slot ring and
-//                          dO_i into its own slot.
-//               warp 1     tcgen05 issuer and TMEM owner.  TMEM columns:
-//                          A = [0,128): S^T, then P^T (16-bit) in [0,64)
-//                          B = [128,256): dP^T, then dS^T in [0,64), then dQ_i
+//   bwd_main  a persistent grid (at most one CTA per SM, 512 threads): each
+//             CTA claims work units (key/value tile j of one head, and of one
+//             sequence in a packed batch) one after another from a counter
+//             in the workspace, in increasing unit order, and broadcasts each
+//             claim to its roles through a two-slot ring in shared memory:
+//               warp 0     TMA producer: claims the next unit, then K_j, V_j
+//                          (once the previous unit's products are done with
+//                          the old ones), Q_i (+ the per-query rows of tile i)
+//                          into a 2-slot ring and dO_i into its own slot.
+//               warp 1     tcgen05 issuer and TMEM owner.  Two 128-column
+//                          regions swap roles every step g: X(g) takes S^T(g),
+//                          which the P warps turn into P^T (16-bit, columns
+//                          [64h, 64h + 32) for query half h) and then dS^T
+//                          (columns [64h + 32, 64h + 64)); Y(g) takes dP^T(g).
+//                          Per step:
+//                            dV  += P^T dO_i               (A = P^T in X)
+//                            S^T(g+1) = K_j Q_{i+1}^T -> Y (as soon as the dS
+//                                       warps have read dP^T(g) out of Y), plus
+//                                       one K step that adds -LSE / scale
+//                            dK  += dS^T Q_i               (A = dS^T in X)
+//                            dQ_i = dS K_j -> X            (A = dS in smem)
+//                            dP^T(g+1) = V_j dO_{i+1}^T -> X (after dQ_i has
+//                                       been drained), plus one K step that
+//                                       adds -D
+//                          so the next step's exponentials start while dK,
+//                          dQ and the next dP^T are on the tensor core.
 //                          dV [256,256+D), dK [256+D,256+2D).
-//                          Issue order for query tile i (one step):
-//                            dV  += P^T dO_i          (A = P^T in TMEM)
-//                            S^T(i+1) = K_j Q_{i+1}^T  -> A, plus one K step
-//                                       that adds -LSE / scale per query
-//                            dK  += dS^T Q_i          (A = dS^T in TMEM)
-//                            dQ_i = dS K_j            (A = dS in smem) -> B
-//                            dP^T(i+1) = V_j dO_{i+1}^T -> B (after dQ_i left
-//                                       TMEM), plus one K step that adds -D
-//                          so the exponentials of tile i+1 run while the
-//                          tensor core does dK_i, dQ_i and dP^T(i+1).
 //               warps 4-11 one thread per key row and half of the query
 //                          columns (warps 4-7 queries 0-63, 8-11 queries
 //                          64-127).  P phase: P^T = exp2(S'^T*scale*log2e)
 //                          (S' already holds -LSE/scale), kept as 16-bit
-//                          pairs in registers and written to TMEM A.  dS
-//                          phase: dS^T = P^T dP'^T (dP' already holds -D) to
-//                          TMEM B and, as the MN-major A operand of
-//                          dQ = dS K, to shared memory.  At the end: dV and
-//                          scale*dK rows to global memory.
+//                          pairs in registers and written to X.  dS phase:
+//                          read dP'^T (it already holds -D) out of Y, then
+//                          dS^T = P^T dP'^T to X and, as the MN-major A
+//                          operand of dQ = dS K, to shared memory.  After a
+//                          unit's last step: its dV and scale*dK rows to global
+//                          memory.
 //               warps 12-15 one thread per query row: move dQ_i from TMEM to
 //                          a per-warp 128-byte-swizzled staging buffer and add
 //                          it to the fp32 accumulator with TMA bulk reductions
 //                          (cp.reduce.async.bulk.tensor .add); under
-//                          deterministic mode the key tiles take turns (in
-//                          increasing j) to issue those reductions for tile i.
+//                          deterministic mode the key tiles take turns to
+//                          issue those reductions for tile i, from the highest
+//                          j down (the order in which they reach tile i), and
+//                          the units are numbered so that every key tile is
+//                          claimed after the one whose turn precedes it: that
+//                          one is always held by a running CTA, whatever order
+//                          the hardware starts CTAs in.
 //   bwd_post  dQ = scale * accumulator, rounded to the input dtype.
 // Causal: key tile j only meets query tiles i >= j; only the diagonal tile
 // is masked element-wise.  Packed batches ([H, T, D], cu_seqlens): every
@@ -61,6 +75,12 @@
 
 #include "sm100.cuh"
 
+// Timeline hooks: BWD_TRACE(condition, slot) records a clock at a point of
+// the pipeline in builds that define it; it compiles to nothing otherwise.
+#ifndef BWD_TRACE
+#define BWD_TRACE(cond, slot) ((void)0)
+#endif
+
 namespace fa {
 
 struct BwdParams {
@@ -71,12 +91,14 @@ struct BwdParams {
                            //   0-8: -LSE*log2(e) in three parts (part k % 3 in column k),
                            //   9-11: -D_i in three parts, 12-15: 0; padding rows -1e30 and 0
   uint32_t* sem;           // [heads, nseq, n_q] ordering counters (deterministic mode)
+  uint32_t* ticket;        // next unit to claim (zeroed by bwd_pre)
   const int* cu_seqlens;   // packed batch only: device int32 [nseq + 1]
   int heads;               // dense: B*H, packed: H
   int S;                   // dense: S, packed: max_seqlen
   int rows;                // rows of one head slice in memory: S or total
   int nseq;                // dense: 1
   int S_pad, n_q;          // ceil(S / 128) * 128, ceil(S / 128)
+  int units;               // unit numbers: groups of kBwdGroup slices x n_q key tiles (some empty)
   float scale, scale_log2;
   int deterministic;
   Dropout drop;            // DROPOUT instances only
@@ -96,9 +118,11 @@ struct BwdCfg {
   static constexpr uint32_t CT_OFF = STG_OFF + 4 * 4096;         // 2 slots x per-query rows (128 x 32 B)
   static constexpr uint32_t ONES_OFF = CT_OFF + 2 * 4096;         // the two constant key-side rows (128 x 32 B)
   static constexpr uint32_t BAR_OFF = ONES_OFF + 2 * 4096;
-  // kv_full q_full[2] q_empty[2] do_full do_empty s_full dp_full p_full ds_full
-  // dq_full dq_empty dkv_full drain dq_done
-  static constexpr int NBAR = 17;
+  // kv_full kv_empty q_full[2] q_empty[2] do_full do_empty s_full dp_full
+  // p_full dp_taken ds_full dq_full dq_empty dkv_full drain dq_done
+  // unit_full[2] unit_empty[2]
+  static constexpr int NBAR = 22;
+  // then the TMEM address and the two-slot unit ring
   static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
   static constexpr uint32_t TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
 };
@@ -109,8 +133,49 @@ constexpr int kBwdGroup = 4;
 enum : uint32_t {
   BWD_SITE_PROD = 0x200, BWD_SITE_KV = 0x201, BWD_SITE_Q = 0x202, BWD_SITE_DO = 0x203, BWD_SITE_P = 0x204,
   BWD_SITE_DS = 0x205, BWD_SITE_DQE = 0x206, BWD_SITE_S = 0x207, BWD_SITE_DP = 0x208, BWD_SITE_DQF = 0x209,
-  BWD_SITE_DKV = 0x20a, BWD_SITE_SEM = 0x20b, BWD_SITE_DRAIN = 0x20c, BWD_SITE_STAT = 0x20d
+  BWD_SITE_DKV = 0x20a, BWD_SITE_SEM = 0x20b, BWD_SITE_DRAIN = 0x20c, BWD_SITE_STAT = 0x20d, BWD_SITE_UNIT = 0x20e,
+  BWD_SITE_TAKEN = 0x20f
 };
+
+// One work unit: key/value tile j of one (sequence, head) slice, which meets
+// query tiles i_begin .. n_q - 1 of its sequence.
+struct BwdUnit {
+  int j, seq, head, row_base, seq_len, n_q, i_begin, n_steps;
+};
+
+// Unit u as its key tile and slice.  Unit numbers walk the (sequence, head)
+// slices in groups of kBwdGroup and, inside a group, ascending j (longest
+// causal work first), so only a few slices are live at a time and their fp32
+// dQ accumulators and Q/K/V/dO tiles stay in L2, where the dQ reductions run
+// about twice as fast as against device memory.  False for a number past the
+// end of a shorter last group or of its sequence; those are skipped.
+template <bool CAUSAL, bool VARLEN>
+__device__ __forceinline__ bool bwd_decode(const BwdParams& p, int u, BwdUnit& x) {
+  const int slices = p.nseq * p.heads;
+  const int group = u / (kBwdGroup * p.n_q);
+  const int rg = u - group * (kBwdGroup * p.n_q);
+  const int gsize = min(kBwdGroup, slices - group * kBwdGroup);
+  const int jr = rg / gsize;
+  if (jr >= p.n_q) return false;
+  // deterministic mode takes a slice's key tiles from the last one down: its
+  // query tiles receive their dQ parts in that order, which is the order in
+  // which the key tiles reach them
+  x.j = p.deterministic ? p.n_q - 1 - jr : jr;
+  const int slice = group * kBwdGroup + (rg - jr * gsize);
+  x.seq = slice / p.heads;
+  x.head = slice - x.seq * p.heads;
+  x.row_base = 0;
+  x.seq_len = p.S;
+  if constexpr (VARLEN) {
+    x.row_base = p.cu_seqlens[x.seq];
+    x.seq_len = p.cu_seqlens[x.seq + 1] - x.row_base;
+  }
+  if (128 * x.j >= x.seq_len) return false;
+  x.n_q = (x.seq_len + 127) / 128;
+  x.i_begin = CAUSAL ? x.j : 0;
+  x.n_steps = x.n_q - x.i_begin;
+  return true;
+}
 
 // ---------------------------------------------------------------------------
 // bwd_pre: one group of D/8 lanes per row, 16-byte loads, shuffle reduction.
@@ -186,6 +251,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict
   for (long long i = gtid; i < n4; i += nthreads) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   const long long ns = (long long)p.heads * p.nseq * p.n_q;
   for (long long i = gtid; i < ns; i += nthreads) p.sem[i] = 0u;
+  if (gtid == 0) *p.ticket = 0u;
 }
 
 // ---------------------------------------------------------------------------
@@ -242,65 +308,49 @@ __global__ void __launch_bounds__(512, 1)
                     const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_cols,
                     const BwdParams p) {
   using C = BwdCfg<D>;
-  // work unit: (key/value tile j, sequence, head).  Blocks walk groups of
-  // kBwdGroup (sequence, head) slices; inside a group, ascending j (longest
-  // causal work first).  Only a few slices are live at a time, so their fp32
-  // dQ accumulators and Q/K/V/dO tiles stay in L2, where the dQ reductions
-  // run about twice as fast as against device memory.
-  const int units = p.nseq * p.heads;
-  const int group = blockIdx.x / (kBwdGroup * p.n_q);
-  const int rg = blockIdx.x - group * (kBwdGroup * p.n_q);
-  const int gsize = min(kBwdGroup, units - group * kBwdGroup);
-  const int j = rg / gsize;
-  if (j >= p.n_q) return;  // the last group may be smaller than kBwdGroup
-  const int unit = group * kBwdGroup + (rg - j * gsize);
-  const int seq = unit / p.heads;
-  const int head = unit - seq * p.heads;
-  int row_base = 0, seq_len = p.S;  // first token row and length of this sequence
-  if constexpr (VARLEN) {
-    row_base = p.cu_seqlens[seq];
-    seq_len = p.cu_seqlens[seq + 1] - row_base;
-  }
-  if (128 * j >= seq_len) return;  // uniform over the CTA, before any set-up
-  const int n_q = (seq_len + 127) / 128;
-  const int i_begin = CAUSAL ? j : 0;
-  const int n_steps = n_q - i_begin;
-  const int kv_row0 = 128 * j;  // inside the sequence
-  const size_t stat_row0 = ((size_t)head * p.nseq + seq) * p.S_pad;  // padded statistics of this sequence
-
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-  uint64_t* kv_full = bars;
-  uint64_t* q_full = bars + 1;    // [2]
-  uint64_t* q_empty = bars + 3;   // [2]
-  uint64_t* do_full = bars + 5;
-  uint64_t* do_empty = bars + 6;
-  uint64_t* s_full = bars + 7;
-  uint64_t* dp_full = bars + 8;
-  uint64_t* p_full = bars + 9;
-  uint64_t* ds_full = bars + 10;
-  uint64_t* dq_full = bars + 11;
-  uint64_t* dq_empty = bars + 12;
-  uint64_t* dkv_full = bars + 13;
-  uint64_t* drain = bars + 14;
-  uint64_t* dq_done = bars + 15;
+  uint64_t* kv_full = bars;        // K_j, V_j loaded
+  uint64_t* kv_empty = bars + 1;   // the unit's last products are done with K_j, V_j
+  uint64_t* q_full = bars + 2;     // [2]
+  uint64_t* q_empty = bars + 4;    // [2]
+  uint64_t* do_full = bars + 6;
+  uint64_t* do_empty = bars + 7;
+  uint64_t* s_full = bars + 8;     // S^T(g) in X(g)
+  uint64_t* dp_full = bars + 9;    // dP^T(g) in Y(g)
+  uint64_t* p_full = bars + 10;    // P^T(g) written (256 P/dS threads)
+  uint64_t* dp_taken = bars + 11;  // dP^T(g) read out of Y(g) (256 P/dS threads)
+  uint64_t* ds_full = bars + 12;   // dS(g) in X(g) and in shared memory (256 P/dS threads)
+  uint64_t* dq_full = bars + 13;   // dQ(g) in X(g)
+  uint64_t* dq_empty = bars + 14;  // dQ(g) read out of X(g) (128 dQ threads)
+  uint64_t* dkv_full = bars + 15;  // the unit's dV and dK are final
+  uint64_t* drain = bars + 16;
+  uint64_t* dq_done = bars + 17;   // deterministic mode: this tile's dQ reductions performed (128 dQ threads)
+  uint64_t* unit_full = bars + 18;   // [2] a claimed unit number is in the ring
+  uint64_t* unit_empty = bars + 20;  // [2] every role has read it (one lane of each of 13 warps)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBAR);
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(tmem_holder + 1);  // [2]
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
 
+  BWD_TRACE(threadIdx.x == 0, 4000);
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+      mbar_init(&unit_full[i], 1);
+      mbar_init(&unit_empty[i], 13);
     }
     mbar_init(do_full, 1);
     mbar_init(do_empty, 1);
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_full, 256);
+    mbar_init(dp_taken, 256);
     mbar_init(ds_full, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
@@ -338,6 +388,20 @@ __global__ void __launch_bounds__(512, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  // Every role but the producer takes the k-th claimed unit from the ring
+  // (-1 ends the list); one lane per warp reports that it has read it.
+  auto next_unit = [&](int k, int& u) -> bool {
+    const int slot = k & 1;
+    if (!__all_sync(0xffffffffu, mbar_wait(&unit_full[slot], (k >> 1) & 1, BWD_SITE_UNIT))) return false;
+    u = unit_ring[slot];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&unit_empty[slot]);
+    return true;
+  };
+  // TMEM region that holds S^T / P^T / dS^T at step g (the other one holds
+  // dP^T and then dQ)
+  auto region_x = [](uint32_t g) -> uint32_t { return (g & 1) ? C::TM_B : C::TM_A; };
+
   // register split over 512 threads launched with 128 each (65536):
   // 128 x 56 (warps 0-3) + 256 x 136 (P/dS) + 128 x 176 (dQ) = 64512.
   // Each warpgroup changes its budget inside its own branch.
@@ -351,36 +415,51 @@ __global__ void __launch_bounds__(512, 1)
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
       tma_prefetch_desc(&tm_cols);
-      mbar_expect_tx(kv_full, 2 * C::TILE);
-      for (int c = 0; c < C::CH; ++c) {
-        tma_load_3d(smem + C::K_OFF + c * C::CHUNK, &tm_k, kv_full, c * 64, row_base + kv_row0, head);
-        tma_load_3d(smem + C::V_OFF + c * C::CHUNK, &tm_v, kv_full, c * 64, row_base + kv_row0, head);
-      }
+      uint32_t g = 0, kc = 0;  // query steps and units loaded so far
       bool ok = true;
-      int q_issued = 0, do_issued = 0;
-      for (int st = 0; st < n_steps && ok; ++st) {
-        const int i = i_begin + st;
-        // Q_i and its LSE / D rows into Q slot st % 2
-        const int qs = st & 1;
-        if (st >= 2 && !(ok = mbar_wait(&q_empty[qs], ((st >> 1) - 1) & 1, BWD_SITE_PROD))) break;
-        mbar_expect_tx(&q_full[qs], C::TILE + 4096u);
-        for (int c = 0; c < C::CH; ++c)
-          tma_load_3d(smem + C::Q_OFF + qs * C::TILE + c * C::CHUNK, &tm_q, &q_full[qs], c * 64,
-                      row_base + 128 * i, head);
-        tma_load_3d(smem + C::CT_OFF + qs * 4096, &tm_cols, &q_full[qs], 0, (int)(stat_row0 + 128 * i), 0);
-        ++q_issued;
-        // dO_i into the dO slot
-        if (st >= 1 && !(ok = mbar_wait(do_empty, (st - 1) & 1, BWD_SITE_PROD))) break;
-        mbar_expect_tx(do_full, C::TILE);
-        for (int c = 0; c < C::CH; ++c)
-          tma_load_3d(smem + C::DO_OFF + c * C::CHUNK, &tm_do, do_full, c * 64, row_base + 128 * i, head);
-        ++do_issued;
+      for (int k = 0; ok; ++k) {
+        // claim the next non-empty unit (numbers past the end claim nothing)
+        int u;
+        BwdUnit x;
+        do {
+          u = (int)atomicAdd(p.ticket, 1u);
+        } while (u < p.units && !bwd_decode<CAUSAL, VARLEN>(p, u, x));
+        const int slot = k & 1;
+        BWD_TRACE(k < 16, 3100 + k);
+        if (k >= 2 && !(ok = mbar_wait(&unit_empty[slot], ((k >> 1) - 1) & 1, BWD_SITE_PROD))) break;
+        unit_ring[slot] = u < p.units ? u : -1;
+        mbar_arrive(&unit_full[slot]);
+        if (u >= p.units) break;
+        // K_j, V_j once the previous unit's products are done with the old ones
+        if (kc > 0 && !(ok = mbar_wait(kv_empty, (kc - 1) & 1, BWD_SITE_PROD))) break;
+        mbar_expect_tx(kv_full, 2 * C::TILE);
+        for (int c = 0; c < C::CH; ++c) {
+          tma_load_3d(smem + C::K_OFF + c * C::CHUNK, &tm_k, kv_full, c * 64, x.row_base + 128 * x.j, x.head);
+          tma_load_3d(smem + C::V_OFF + c * C::CHUNK, &tm_v, kv_full, c * 64, x.row_base + 128 * x.j, x.head);
+        }
+        ++kc;
+        const size_t stat_row0 = ((size_t)x.head * p.nseq + x.seq) * p.S_pad;  // padded statistics of this sequence
+        for (int st = 0; st < x.n_steps && ok; ++st, ++g) {
+          const int i = x.i_begin + st;
+          // Q_i and its LSE / D rows into Q slot g % 2
+          const int qs = g & 1;
+          if (g >= 2 && !(ok = mbar_wait(&q_empty[qs], ((g >> 1) - 1) & 1, BWD_SITE_PROD))) break;
+          mbar_expect_tx(&q_full[qs], C::TILE + 4096u);
+          for (int c = 0; c < C::CH; ++c)
+            tma_load_3d(smem + C::Q_OFF + qs * C::TILE + c * C::CHUNK, &tm_q, &q_full[qs], c * 64,
+                        x.row_base + 128 * i, x.head);
+          tma_load_3d(smem + C::CT_OFF + qs * 4096, &tm_cols, &q_full[qs], 0, (int)(stat_row0 + 128 * i), 0);
+          // dO_i into the dO slot
+          if (g >= 1 && !(ok = mbar_wait(do_empty, (g - 1) & 1, BWD_SITE_PROD))) break;
+          mbar_expect_tx(do_full, C::TILE);
+          for (int c = 0; c < C::CH; ++c)
+            tma_load_3d(smem + C::DO_OFF + c * C::CHUNK, &tm_do, do_full, c * 64, x.row_base + 128 * i, x.head);
+        }
       }
       // no tile copy may still be landing in shared memory at exit
-      mbar_wait(kv_full, 0, BWD_SITE_PROD);
-      for (int u = (q_issued > 2 ? q_issued - 2 : 0); u < q_issued; ++u)
-        mbar_wait(&q_full[u & 1], (u >> 1) & 1, BWD_SITE_PROD);
-      if (do_issued > 0) mbar_wait(do_full, (do_issued - 1) & 1, BWD_SITE_PROD);
+      if (kc > 0) mbar_wait(kv_full, (kc - 1) & 1, BWD_SITE_PROD);
+      for (uint32_t v = (g > 2 ? g - 2 : 0); v < g; ++v) mbar_wait(&q_full[v & 1], (v >> 1) & 1, BWD_SITE_PROD);
+      if (g > 0) mbar_wait(do_full, (g - 1) & 1, BWD_SITE_PROD);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -398,7 +477,7 @@ __global__ void __launch_bounds__(512, 1)
     const uint64_t qMN = make_sdesc(smem_addr(smem + C::Q_OFF), C::CHUNK, 1024);  // Q slot 0 as B of dK
     const uint64_t doK = make_sdesc(smem_addr(smem + C::DO_OFF), 16, 1024);
     const uint64_t doMN = make_sdesc(smem_addr(smem + C::DO_OFF), C::CHUNK, 1024);
-    const uint64_t dsMN = make_sdesc(smem_addr(smem + C::DS_OFF), C::CHUNK, 1024);
+    const uint64_t dsMN = make_sdesc(smem_addr(smem + C::DS_OFF), C::CHUNK, 1024);  // dS as A of dQ (MN-major)
     const uint64_t onesL = make_sdesc_sw32(smem_addr(smem + C::ONES_OFF));         // adds -LSE / scale
     const uint64_t onesD = make_sdesc_sw32(smem_addr(smem + C::ONES_OFF + 4096));  // adds -D
     const uint64_t ctK = make_sdesc_sw32(smem_addr(smem + C::CT_OFF));              // per-query rows, slot 0
@@ -412,64 +491,91 @@ __global__ void __launch_bounds__(512, 1)
       }
     };
     // acc += A(TMEM, 16-bit pairs) * B (MN-major), K = 128 queries.  Queries
-    // 0-63 sit in the first 32 columns of the A region, queries 64-127 in
-    // columns 64-95 (each half is written by the warpgroup that read those
-    // score columns).
+    // 0-63 sit in columns a_col .. a_col + 31, queries 64-127 in columns
+    // a_col + 64 .. a_col + 95 (each half is written by the warpgroup that
+    // read those score columns).
     auto ts_product = [&](uint32_t d_col, uint32_t a_col, uint64_t b, uint32_t acc) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
         mma_ts_e(tmem + d_col, tmem + a_col + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), desc_add(b, kk * 2048), ID_TS,
                  kk > 0 ? 1u : acc, e);
     };
-    bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0, BWD_SITE_KV) && mbar_wait(&q_full[0], 0, BWD_SITE_Q) &&
-                                          mbar_wait(do_full, 0, BWD_SITE_DO));
-    if (ok) {
-      tc_fence_after();
-      kk_product(C::TM_A, kK, qK);  // S^T(0), then - LSE / scale
-      mma_ss_e(tmem + C::TM_A, onesL, ctK, ID_AUG, 1u, e);
-      mma_commit_e(s_full, e);
-      kk_product(C::TM_B, vK, doK);  // dP^T(0), then - D
-      mma_ss_e(tmem + C::TM_B, onesD, ctK, ID_AUG, 1u, e);
-      mma_commit_e(dp_full, e);
-    }
-    for (int st = 0; st < n_steps && ok; ++st) {
-      const int qs = st & 1;
-      const uint32_t acc = st > 0 ? 1u : 0u;
-      // dV += P^T dO_i
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_full, st & 1, BWD_SITE_P)))) break;
-      tc_fence_after();
-      ts_product(C::TM_DV, C::TM_A, doMN, acc);
-      mma_commit_e(do_empty, e);
-      // S^T(i+1) into A (P^T(i) has been read by the products above)
-      const bool more = st + 1 < n_steps;
-      if (more) {
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&q_full[qs ^ 1], ((st + 1) >> 1) & 1, BWD_SITE_Q)))) break;
+    uint32_t g = 0, kc = 0;  // query steps and units so far
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      int u;
+      if (!(ok = next_unit(k, u)) || u < 0) break;
+      BwdUnit x;
+      bwd_decode<CAUSAL, VARLEN>(p, u, x);
+      BWD_TRACE(lane == 0 && k < 16, 3000 + 2 * k);
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(kv_full, kc & 1, BWD_SITE_KV)))) break;
+      BWD_TRACE(lane == 0 && k < 16, 3000 + 2 * k + 1);
+      ++kc;
+      // first step of the unit: S^T(g) into X(g), dP^T(g) into Y(g) = X(g - 1),
+      // which still holds dQ(g - 1) until the dQ warps have drained it
+      {
+        const int qs = g & 1;
+        const uint32_t X = region_x(g), Y = X ^ (C::TM_A ^ C::TM_B);
+        ok = mbar_wait(&q_full[qs], (g >> 1) & 1, BWD_SITE_Q) && mbar_wait(do_full, g & 1, BWD_SITE_DO);
+        if (ok && g > 0) ok = mbar_wait(dq_empty, (g - 1) & 1, BWD_SITE_DQE);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
         tc_fence_after();
-        kk_product(C::TM_A, kK, desc_add(qK, (qs ^ 1) * C::TILE));
-        mma_ss_e(tmem + C::TM_A, onesL, desc_add(ctK, (qs ^ 1) * 4096), ID_AUG, 1u, e);
+        kk_product(X, kK, desc_add(qK, qs * C::TILE));  // S^T(g), then - LSE / scale
+        mma_ss_e(tmem + X, onesL, desc_add(ctK, qs * 4096), ID_AUG, 1u, e);
         mma_commit_e(s_full, e);
-      }
-      // dK += dS^T Q_i
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_full, st & 1, BWD_SITE_DS)))) break;
-      tc_fence_after();
-      ts_product(C::TM_DK, C::TM_B, desc_add(qMN, qs * C::TILE), acc);
-      mma_commit_e(&q_empty[qs], e);
-      // dQ_i = dS K_j into B  (A = dS MN-major in smem, B = K MN-major)
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ss_e(tmem + C::TM_B, desc_add(dsMN, kk * 2048), desc_add(kMN, kk * 2048), ID_DQ, kk > 0 ? 1u : 0u, e);
-      mma_commit_e(dq_full, e);
-      // dP^T(i+1) into B once dQ_i has been drained
-      if (more) {
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_empty, st & 1, BWD_SITE_DQE)))) break;
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(do_full, (st + 1) & 1, BWD_SITE_DO)))) break;
-        tc_fence_after();
-        kk_product(C::TM_B, vK, doK);
-        mma_ss_e(tmem + C::TM_B, onesD, desc_add(ctK, (qs ^ 1) * 4096), ID_AUG, 1u, e);
+        kk_product(Y, vK, doK);  // dP^T(g), then - D
+        mma_ss_e(tmem + Y, onesD, desc_add(ctK, qs * 4096), ID_AUG, 1u, e);
         mma_commit_e(dp_full, e);
       }
+      for (int st = 0; st < x.n_steps && ok; ++st, ++g) {
+        const int qs = g & 1;
+        const uint32_t X = region_x(g), Y = X ^ (C::TM_A ^ C::TM_B);
+        const uint32_t acc = st > 0 ? 1u : 0u;
+        const bool more = st + 1 < x.n_steps;
+        // dV += P^T dO_i (dO_i is not read again: dP^T(g) came before)
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_full, g & 1, BWD_SITE_P)))) break;
+        BWD_TRACE(lane == 0 && g < 200, g * 8);
+        tc_fence_after();
+        ts_product(C::TM_DV, X, doMN, acc);
+        mma_commit_e(do_empty, e);
+        // S^T(g+1) into Y as soon as the dS warps have read dP^T(g) out of it
+        if (more) {
+          ok = mbar_wait(dp_taken, g & 1, BWD_SITE_TAKEN) && mbar_wait(&q_full[qs ^ 1], ((g + 1) >> 1) & 1, BWD_SITE_Q);
+          if (!(ok = __all_sync(0xffffffffu, ok))) break;
+          tc_fence_after();
+          BWD_TRACE(lane == 0 && g < 200, g * 8 + 1);
+          kk_product(Y, kK, desc_add(qK, (qs ^ 1) * C::TILE));
+          mma_ss_e(tmem + Y, onesL, desc_add(ctK, (qs ^ 1) * 4096), ID_AUG, 1u, e);
+          mma_commit_e(s_full, e);
+        }
+        // dK += dS^T Q_i (A = dS^T in X; Q_i is not read again)
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(ds_full, g & 1, BWD_SITE_DS)))) break;
+        BWD_TRACE(lane == 0 && g < 200, g * 8 + 2);
+        tc_fence_after();
+        ts_product(C::TM_DK, X + 32, desc_add(qMN, qs * C::TILE), acc);
+        mma_commit_e(&q_empty[qs], e);
+        // dQ_i = dS K_j into X  (A = dS MN-major in smem, B = K MN-major),
+        // after dK has read dS^T out of X
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss_e(tmem + X, desc_add(dsMN, kk * 2048), desc_add(kMN, kk * 2048), ID_DQ, kk > 0 ? 1u : 0u, e);
+        mma_commit_e(dq_full, e);
+        BWD_TRACE(lane == 0 && g < 200, g * 8 + 3);
+        // dP^T(g+1) into X once dQ_i has been drained
+        if (more) {
+          ok = mbar_wait(dq_empty, g & 1, BWD_SITE_DQE) && mbar_wait(do_full, (g + 1) & 1, BWD_SITE_DO);
+          if (!(ok = __all_sync(0xffffffffu, ok))) break;
+          BWD_TRACE(lane == 0 && g < 200, g * 8 + 4);
+          tc_fence_after();
+          kk_product(X, vK, doK);
+          mma_ss_e(tmem + X, onesD, desc_add(ctK, (qs ^ 1) * 4096), ID_AUG, 1u, e);
+          mma_commit_e(dp_full, e);
+        }
+      }
+      if (!ok) break;
+      mma_commit_e(kv_empty, e);  // K_j, V_j may be replaced
+      mma_commit_e(dkv_full, e);  // this unit's dV, dK are final
     }
-    mma_commit_e(dkv_full, e);
     mma_commit_e(drain, e);
     mbar_wait(drain, 0, BWD_SITE_DRAIN);
     __syncwarp();
@@ -483,177 +589,197 @@ __global__ void __launch_bounds__(512, 1)
     const int half = (warp - 4) >> 2;
     const int r = (threadIdx.x - 128) & 127;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t tA = tmem + lane_off + C::TM_A, tB = tmem + lane_off + C::TM_B;
-    const int kv = kv_row0 + r;
-    const bool kv_valid = kv < seq_len;
     const float sl2 = p.scale_log2;
     uint8_t* ds_smem = smem + C::DS_OFF;
+    uint32_t g = 0, ucnt = 0;  // query steps and units so far
     bool ok = true;
-    for (int st = 0; st < n_steps; ++st) {
-      const int i = i_begin + st;
-      const int qs = st & 1;
-      ok = mbar_wait(s_full, st & 1, BWD_SITE_S) && mbar_wait(&q_full[qs], (st >> 1) & 1, BWD_SITE_STAT);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      // visible queries of this key row in tile i: q >= kv under the causal mask
-      const int qlo = (CAUSAL && i == j) ? r : 0;
-      const bool masked = qlo > 64 * half || !kv_valid;  // some column of this half is invisible
-      // ---- P phase (score columns 64*half .. +63): the scores already hold
-      // -LSE / scale (extra K step), so P^T = 2^(S'^T scale log2 e)
-      uint32_t sv[2][32];
-      tmem_ld32(tA + 64 * half, sv[0]);
-      tmem_ld32(tA + 64 * half + 32, sv[1]);
-      tmem_ld_wait(sv[0]);
-      tmem_ld_wait(sv[1]);
-      const uint64_t sl2x2 = f2(sl2, sl2);
-      uint32_t pk[32];  // P pairs rounded to 16 bits (the products' and dS's P)
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int c = 64 * half + 2 * e;
-        const uint32_t* src = sv[e >> 4] + 2 * (e & 15);
-        float p0, p1;
-        f2split(fmul2(f2(__uint_as_float(src[0]), __uint_as_float(src[1])), sl2x2), p0, p1);
-        p0 = ex2(p0);
-        p1 = ex2(p1);
-        if (masked) {
-          if (c < qlo || !kv_valid) p0 = 0.f;
-          if (c + 1 < qlo || !kv_valid) p1 = 0.f;
-        }
-        pk[e] = pack2<BF16>(p0, p1);
-      }
-      // dropout keep masks of the 64 query columns: bit e of keep_lo / keep_hi
-      // for queries 2e and 2e + 1 of this half.  One Philox call covers query
-      // pair e x key quad (4m .. 4m + 3), 16 bits per element, and a key quad
-      // sits in four consecutive lanes: lane 4m + c draws query pairs
-      // 8c .. 8c + 7, and each lane hands every other lane of its quad that
-      // lane's two 16-bit values (XOR shuffles over the quad).
-      uint32_t keep_lo = 0xFFFFFFFFu, keep_hi = 0xFFFFFFFFu;
-      if constexpr (DROPOUT) {
-        const uint32_t c4 = lane & 3u, th = p.drop.thresh;
-        const uint32_t keyquad = (uint32_t)kv >> 2, qp0 = (uint32_t)(128 * i + 64 * half) >> 1;
-        keep_lo = keep_hi = 0u;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint4 w = philox4x32_10(make_uint4(keyquad, qp0 + 8 * c4 + k, (uint32_t)head, p.drop.offset),
-                                        p.drop.seed_lo, p.drop.seed_hi);
-          // key 4m + t: word (t >> 1) for the even query, 2 + (t >> 1) for
-          // the odd one; half t & 1 of each; packed (even, odd) as 2 x 16 bits
-          auto vals_for = [&w](uint32_t t) -> uint32_t {
-            const uint32_t we = (t & 2u) ? w.y : w.x, wo = (t & 2u) ? w.w : w.z;
-            return (t & 1u) ? ((we >> 16) | (wo & 0xFFFF0000u)) : ((we & 0xFFFFu) | (wo << 16));
-          };
-#pragma unroll
-          for (uint32_t d = 0; d < 4; ++d) {
-            const uint32_t v = d == 0 ? vals_for(c4) : __shfl_xor_sync(0xffffffffu, vals_for(c4 ^ d), (int)d);
-            const uint32_t e = 8u * (c4 ^ d) + (uint32_t)k;  // query pair drawn by lane c4 ^ d
-            keep_lo |= ((v & 0xFFFFu) < th ? 1u : 0u) << e;
-            keep_hi |= ((v >> 16) < th ? 1u : 0u) << e;
-          }
-        }
-      }
-      // P^T pairs go to columns [64*half, 64*half + 32) of A (inside this
-      // half's own score columns, already read); with dropout the dV operand
-      // is P * M (dV is scaled by s = 1 / keep probability at the end)
-      if constexpr (DROPOUT) {
-        uint32_t pd[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          pd[e] = pk[e] & (((keep_lo >> e) & 1u ? 0x0000FFFFu : 0u) | ((keep_hi >> e) & 1u ? 0xFFFF0000u : 0u));
-        tmem_st32(tA + 64 * half, pd);
-      } else {
-        tmem_st32(tA + 64 * half, pk);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(p_full);
-      // ---- dS phase: dS^T = P^T (dP^T - D), P as rounded for the products;
-      // dP^T already holds -D (extra K step)
-      ok = __all_sync(0xffffffffu, mbar_wait(dp_full, st & 1, BWD_SITE_DP));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t dv[2][32];
-      tmem_ld32(tB + 64 * half, dv[0]);
-      tmem_ld32(tB + 64 * half + 32, dv[1]);
-      tmem_ld_wait(dv[0]);
-      tmem_ld_wait(dv[1]);
-      uint32_t dd[32];
-      if constexpr (DROPOUT) {
-        // dP'^T = dPd^T - D (extra K step).  Kept: dS = P (dPd s - D)
-        // = P (dP' s + D (s - 1)); dropped: dS = -P D  (s = 1 / keep probability).
-        // D_i of the query rows comes from their per-query row (-D in three
-        // bf16 parts, columns 9-11) in shared memory.
-        const uint8_t* ct = smem + C::CT_OFF + qs * 4096;
-        const float rp = p.drop.scale, rp1 = p.drop.scale - 1.f;
+    for (int k = 0; ok; ++k) {
+      int u;
+      if (!(ok = next_unit(k, u)) || u < 0) break;
+      BwdUnit x;
+      bwd_decode<CAUSAL, VARLEN>(p, u, x);
+      const int kv = 128 * x.j + r;  // key row inside the sequence
+      const bool kv_valid = kv < x.seq_len;
+      for (int st = 0; st < x.n_steps; ++st, ++g) {
+        const int i = x.i_begin + st;
+        const int qs = g & 1;
+        const uint32_t X = region_x(g), Y = X ^ (C::TM_A ^ C::TM_B);
+        const uint32_t tX = tmem + lane_off + X, tY = tmem + lane_off + Y;
+        ok = mbar_wait(s_full, g & 1, BWD_SITE_S) && mbar_wait(&q_full[qs], (g >> 1) & 1, BWD_SITE_STAT);
+        ok = __all_sync(0xffffffffu, ok);
+        const bool tw = warp == 4 && lane == 0 && g < 200;
+        BWD_TRACE(tw, 1600 + 4 * g);
+        if (!ok) break;
+        tc_fence_after();
+        // visible queries of this key row in tile i: q >= kv under the causal mask
+        const int qlo = (CAUSAL && i == x.j) ? r : 0;
+        const bool masked = qlo > 64 * half || !kv_valid;  // some column of this half is invisible
+        // ---- P phase (score columns 64*half .. +63): the scores already hold
+        // -LSE / scale (extra K step), so P^T = 2^(S'^T scale log2 e)
+        uint32_t sv[2][32];
+        tmem_ld32(tX + 64 * half, sv[0]);
+        tmem_ld32(tX + 64 * half + 32, sv[1]);
+        tmem_ld_wait(sv[0]);
+        tmem_ld_wait(sv[1]);
+        const uint64_t sl2x2 = f2(sl2, sl2);
+        uint32_t pk[32];  // P pairs rounded to 16 bits (the products' and dS's P)
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const uint32_t* src = dv[e >> 4] + 2 * (e & 15);
-          float dq[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const uint32_t qrow = (uint32_t)(64 * half + 2 * e + u);
-            const uint2 c = *reinterpret_cast<const uint2*>(ct + swz32(qrow * 32u + 16u));
-            dq[u] = -(__uint_as_float(c.x & 0xFFFF0000u) + __uint_as_float(c.y << 16) +
-                      __uint_as_float(c.y & 0xFFFF0000u));
+          const int c = 64 * half + 2 * e;
+          const uint32_t* src = sv[e >> 4] + 2 * (e & 15);
+          float p0, p1;
+          f2split(fmul2(f2(__uint_as_float(src[0]), __uint_as_float(src[1])), sl2x2), p0, p1);
+          p0 = ex2(p0);
+          p1 = ex2(p1);
+          if (masked) {
+            if (c < qlo || !kv_valid) p0 = 0.f;
+            if (c + 1 < qlo || !kv_valid) p1 = 0.f;
           }
-          const float2 pw = unpack2<BF16>(pk[e]);
-          const float a = pw.x * (((keep_lo >> e) & 1u) ? fmaf(__uint_as_float(src[0]), rp, dq[0] * rp1) : -dq[0]);
-          const float b = pw.y * (((keep_hi >> e) & 1u) ? fmaf(__uint_as_float(src[1]), rp, dq[1] * rp1) : -dq[1]);
-          dd[e] = pack2<BF16>(a, b);
+          pk[e] = pack2<BF16>(p0, p1);
         }
-      } else {
+        // dropout keep masks of the 64 query columns: bit e of keep_lo / keep_hi
+        // for queries 2e and 2e + 1 of this half.  One Philox call covers query
+        // pair e x key quad (4m .. 4m + 3), 16 bits per element, and a key quad
+        // sits in four consecutive lanes: lane 4m + c draws query pairs
+        // 8c .. 8c + 7, and each lane hands every other lane of its quad that
+        // lane's two 16-bit values (XOR shuffles over the quad).
+        uint32_t keep_lo = 0xFFFFFFFFu, keep_hi = 0xFFFFFFFFu;
+        if constexpr (DROPOUT) {
+          const uint32_t c4 = lane & 3u, th = p.drop.thresh;
+          const uint32_t keyquad = (uint32_t)kv >> 2, qp0 = (uint32_t)(128 * i + 64 * half) >> 1;
+          keep_lo = keep_hi = 0u;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const uint32_t* src = dv[e >> 4] + 2 * (e & 15);
-          float a, b;
-          f2split(fmul2(widen2<BF16>(pk[e]), f2(__uint_as_float(src[0]), __uint_as_float(src[1]))), a, b);
-          dd[e] = pack2<BF16>(a, b);
+          for (int q = 0; q < 8; ++q) {
+            const uint4 w = philox4x32_10(make_uint4(keyquad, qp0 + 8 * c4 + q, (uint32_t)x.head, p.drop.offset),
+                                          p.drop.seed_lo, p.drop.seed_hi);
+            // key 4m + t: word (t >> 1) for the even query, 2 + (t >> 1) for
+            // the odd one; half t & 1 of each; packed (even, odd) as 2 x 16 bits
+            auto vals_for = [&w](uint32_t t) -> uint32_t {
+              const uint32_t we = (t & 2u) ? w.y : w.x, wo = (t & 2u) ? w.w : w.z;
+              return (t & 1u) ? ((we >> 16) | (wo & 0xFFFF0000u)) : ((we & 0xFFFFu) | (wo << 16));
+            };
+#pragma unroll
+            for (uint32_t d = 0; d < 4; ++d) {
+              const uint32_t v = d == 0 ? vals_for(c4) : __shfl_xor_sync(0xffffffffu, vals_for(c4 ^ d), (int)d);
+              const uint32_t e = 8u * (c4 ^ d) + (uint32_t)q;  // query pair drawn by lane c4 ^ d
+              keep_lo |= ((v & 0xFFFFu) < th ? 1u : 0u) << e;
+              keep_hi |= ((v >> 16) < th ? 1u : 0u) << e;
+            }
+          }
         }
-      }
+        // P^T pairs go to columns [64*half, 64*half + 32) of X (inside this
+        // half's own score columns, already read); with dropout the dV operand
+        // is P * M (dV is scaled by s = 1 / keep probability at the end)
+        if constexpr (DROPOUT) {
+          uint32_t pd[32];
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        // dS row r (key), 32 query columns: MN-major A operand of dQ = dS K,
-        // [key][query] with queries contiguous, 64-query chunk = half, 128-B swizzled
-        const uint32_t base = half * C::CHUNK + r * 128 + ch * 64;
+          for (int e = 0; e < 32; ++e)
+            pd[e] = pk[e] & (((keep_lo >> e) & 1u ? 0x0000FFFFu : 0u) | ((keep_hi >> e) & 1u ? 0xFFFF0000u : 0u));
+          tmem_st32(tX + 64 * half, pd);
+        } else {
+          tmem_st32(tX + 64 * half, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(p_full);
+        BWD_TRACE(tw, 1600 + 4 * g + 1);
+        // ---- dS phase: dS^T = P^T (dP^T - D), P as rounded for the products;
+        // dP^T already holds -D (extra K step).  Once it is in registers Y
+        // is free for the next step's scores.
+        ok = __all_sync(0xffffffffu, mbar_wait(dp_full, g & 1, BWD_SITE_DP));
+        BWD_TRACE(tw, 1600 + 4 * g + 2);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t dv[2][32];
+        tmem_ld32(tY + 64 * half, dv[0]);
+        tmem_ld32(tY + 64 * half + 32, dv[1]);
+        tmem_ld_wait(dv[0]);
+        tmem_ld_wait(dv[1]);
+        tc_fence_before();
+        mbar_arrive(dp_taken);
+        uint32_t dd[32];
+        if constexpr (DROPOUT) {
+          // dP'^T = dPd^T - D (extra K step).  Kept: dS = P (dPd s - D)
+          // = P (dP' s + D (s - 1)); dropped: dS = -P D  (s = 1 / keep probability).
+          // D_i of the query rows comes from their per-query row (-D in three
+          // bf16 parts, columns 9-11) in shared memory.
+          const uint8_t* ct = smem + C::CT_OFF + qs * 4096;
+          const float rp = p.drop.scale, rp1 = p.drop.scale - 1.f;
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4)
-          *reinterpret_cast<uint4*>(ds_smem + swz128(base + v4 * 16)) =
-              make_uint4(dd[16 * ch + 4 * v4], dd[16 * ch + 4 * v4 + 1], dd[16 * ch + 4 * v4 + 2],
-                         dd[16 * ch + 4 * v4 + 3]);
+          for (int e = 0; e < 32; ++e) {
+            const uint32_t* src = dv[e >> 4] + 2 * (e & 15);
+            float dq[2];
+#pragma unroll
+            for (int w2 = 0; w2 < 2; ++w2) {
+              const uint32_t qrow = (uint32_t)(64 * half + 2 * e + w2);
+              const uint2 c = *reinterpret_cast<const uint2*>(ct + swz32(qrow * 32u + 16u));
+              dq[w2] = -(__uint_as_float(c.x & 0xFFFF0000u) + __uint_as_float(c.y << 16) +
+                         __uint_as_float(c.y & 0xFFFF0000u));
+            }
+            const float2 pw = unpack2<BF16>(pk[e]);
+            const float a = pw.x * (((keep_lo >> e) & 1u) ? fmaf(__uint_as_float(src[0]), rp, dq[0] * rp1) : -dq[0]);
+            const float b = pw.y * (((keep_hi >> e) & 1u) ? fmaf(__uint_as_float(src[1]), rp, dq[1] * rp1) : -dq[1]);
+            dd[e] = pack2<BF16>(a, b);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const uint32_t* src = dv[e >> 4] + 2 * (e & 15);
+            float a, b;
+            f2split(fmul2(widen2<BF16>(pk[e]), f2(__uint_as_float(src[0]), __uint_as_float(src[1]))), a, b);
+            dd[e] = pack2<BF16>(a, b);
+          }
+        }
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          // dS row r (key), 32 query columns: MN-major A operand of dQ = dS K,
+          // [key][query] with queries contiguous, 64-query chunk = half, 128-B swizzled
+          const uint32_t base = half * C::CHUNK + r * 128 + ch * 64;
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            *reinterpret_cast<uint4*>(ds_smem + swz128(base + v4 * 16)) =
+                make_uint4(dd[16 * ch + 4 * v4], dd[16 * ch + 4 * v4 + 1], dd[16 * ch + 4 * v4 + 2],
+                           dd[16 * ch + 4 * v4 + 3]);
+        }
+        // dS^T pairs to columns [64*half + 32, 64*half + 64) of X (score
+        // columns this half has read)
+        tmem_st32(tX + 64 * half + 32, dd);
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(ds_full);
+        BWD_TRACE(tw, 1600 + 4 * g + 3);
       }
-      // dS^T pairs to columns [64*half, 64*half + 32) of B (dP columns already read)
-      tmem_st32(tB + 64 * half, dd);
-      fence_proxy_async_smem();
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(ds_full);
-    }
-    // ---- epilogue: dV and scale * dK rows of this key tile
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dkv_full, 0, BWD_SITE_DKV));
-    if (ok) {
+      if (!ok) break;
+      // ---- epilogue: dV and scale * dK rows of this key tile
+      ok = __all_sync(0xffffffffu, mbar_wait(dkv_full, ucnt & 1, BWD_SITE_DKV));
+      BWD_TRACE(warp == 4 && lane == 0 && ucnt < 16, 3200 + ucnt);
+      ++ucnt;
+      if (!ok) break;
       tc_fence_after();
-      const size_t grow = ((size_t)head * p.rows + row_base + kv) * D;
-      {
-        const int which = half;  // half 0 writes dV, half 1 writes scale * dK
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(which ? p.dk : p.dv) + grow);
-        const float mul = which ? p.scale : (DROPOUT ? p.drop.scale : 1.f);
-        const uint32_t col = which ? C::TM_DK : C::TM_DV;
+      const size_t grow = ((size_t)x.head * p.rows + x.row_base + kv) * D;
+      const int which = half;  // half 0 writes dV, half 1 writes scale * dK
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(which ? p.dk : p.dv) + grow);
+      const float mul = which ? p.scale : (DROPOUT ? p.drop.scale : 1.f);
+      const uint32_t col = which ? C::TM_DK : C::TM_DV;
 #pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t ov[32];
-          tmem_ld32(tmem + lane_off + col + 32 * cc, ov);
-          tmem_ld_wait(ov);
-          uint32_t pkk[16];
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t ov[32];
+        tmem_ld32(tmem + lane_off + col + 32 * cc, ov);
+        tmem_ld_wait(ov);
+        uint32_t pkk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pkk[e] = pack2<BF16>(__uint_as_float(ov[2 * e]) * mul, __uint_as_float(ov[2 * e + 1]) * mul);
-          if (kv_valid) {
+        for (int e = 0; e < 16; ++e)
+          pkk[e] = pack2<BF16>(__uint_as_float(ov[2 * e]) * mul, __uint_as_float(ov[2 * e + 1]) * mul);
+        if (kv_valid) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dst[cc * 4 + e] = make_uint4(pkk[4 * e], pkk[4 * e + 1], pkk[4 * e + 2], pkk[4 * e + 3]);
-          }
+          for (int e = 0; e < 4; ++e)
+            dst[cc * 4 + e] = make_uint4(pkk[4 * e], pkk[4 * e + 1], pkk[4 * e + 2], pkk[4 * e + 3]);
         }
       }
+      // the next unit's first dV / dK products overwrite the accumulators only
+      // after this warpgroup has published that unit's first P / dS
+      tc_fence_before();
     }
   } else {
     regs_inc<176>();
@@ -663,72 +789,88 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     uint8_t* stg = smem + C::STG_OFF + wq * 4096;    // 32 rows x 128 B, 128-B swizzled
     if (lane == 0) tma_prefetch_desc(&tm_dq);
-    for (int st = 0; st < n_steps; ++st) {
-      const int i = i_begin + st;
-      if (!__all_sync(0xffffffffu, mbar_wait(dq_full, st & 1, BWD_SITE_DQF))) break;
-      tc_fence_after();
-      uint32_t a[D / 32][32];
+    uint32_t g = 0;  // query steps so far
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      int u;
+      if (!(ok = next_unit(k, u)) || u < 0) break;
+      BwdUnit x;
+      bwd_decode<CAUSAL, VARLEN>(p, u, x);
+      for (int st = 0; st < x.n_steps; ++st, ++g) {
+        const int i = x.i_begin + st;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(dq_full, g & 1, BWD_SITE_DQF)))) break;
+        const bool qw = warp == 12 && lane == 0 && g < 200;
+        BWD_TRACE(qw, 2400 + 3 * g);
+        tc_fence_after();
+        const uint32_t X = region_x(g);
+        uint32_t a[D / 32][32];
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tmem + lane_off + C::TM_B + 32 * cc, a[cc]);
+        for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tmem + lane_off + X + 32 * cc, a[cc]);
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) tmem_ld_wait(a[cc]);
-      tc_fence_before();
-      mbar_arrive(dq_empty);
-      // This tile's fp32 partial: TMEM -> per-warp swizzled staging -> TMA bulk
-      // reduce-add into the accumulator, 32 columns at a time.
-      auto reduce_partial = [&]() {
+        for (int cc = 0; cc < D / 32; ++cc) tmem_ld_wait(a[cc]);
+        tc_fence_before();
+        mbar_arrive(dq_empty);
+        BWD_TRACE(qw, 2400 + 3 * g + 1);
+        // This tile's fp32 partial: TMEM -> per-warp swizzled staging -> TMA bulk
+        // reduce-add into the accumulator, 32 columns at a time.
+        auto reduce_partial = [&]() {
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          if (lane == 0) bulk_wait_read0();  // the previous reduction has read the buffer
-          __syncwarp();
+          for (int cc = 0; cc < D / 32; ++cc) {
+            if (lane == 0) bulk_wait_read0();  // the previous reduction has read the buffer
+            __syncwarp();
 #pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4)
-            *reinterpret_cast<uint4*>(stg + swz128(lane * 128 + v4 * 16)) =
-                make_uint4(a[cc][4 * v4], a[cc][4 * v4 + 1], a[cc][4 * v4 + 2], a[cc][4 * v4 + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_reduce_add_3d(&tm_dq, stg, 32 * cc, row_base + 128 * i + 32 * wq, head);
-            bulk_commit();
-          }
-        }
-      };
-      if (!p.deterministic) {
-        reduce_partial();
-      } else {
-        // Key tiles add into query tile i in increasing j: one poller per warp
-        // waits for our turn, the partial goes in with the same bulk
-        // reductions, and the turn passes on only once they have been
-        // performed, so every element sees its additions in one fixed order.
-        uint32_t* sem = p.sem + ((size_t)head * p.nseq + seq) * p.n_q + i;
-        bool ok = true;
-        if (lane == 0) {
-          if (ld_acquire_gpu(sem) != (uint32_t)j) {
-            const uint64_t t0 = global_ns();
-            while (ld_acquire_gpu(sem) != (uint32_t)j) {
-              if (global_ns() - t0 > kWaitLimitNs) {
-                record_error(DEV_ERR_TIMEOUT, BWD_SITE_SEM);
-                ok = false;
-                break;
-              }
+            for (int v4 = 0; v4 < 8; ++v4)
+              *reinterpret_cast<uint4*>(stg + swz128(lane * 128 + v4 * 16)) =
+                  make_uint4(a[cc][4 * v4], a[cc][4 * v4 + 1], a[cc][4 * v4 + 2], a[cc][4 * v4 + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_reduce_add_3d(&tm_dq, stg, 32 * cc, x.row_base + 128 * i + 32 * wq, x.head);
+              bulk_commit();
             }
           }
-          fence_proxy_async_global();  // our reductions come after the acquire
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (ok) {
+        };
+        if (!p.deterministic) {
           reduce_partial();
+          BWD_TRACE(qw, 2400 + 3 * g + 2);
+        } else {
+          // Key tiles add into query tile i in a fixed order: one poller per
+          // warp waits for our turn, the partial goes in with the same bulk
+          // reductions, and the turn passes on only once they have been
+          // performed, so every element sees its additions in one fixed order.
+          uint32_t* sem = p.sem + ((size_t)x.head * p.nseq + x.seq) * p.n_q + i;
+          // key tiles add into query tile i from the highest down: j = i first
+          // under the causal mask (j = n_q - 1 without it), then j - 1, ...
+          const uint32_t turn = (uint32_t)((CAUSAL ? i : x.n_q - 1) - x.j);
+          bool mine = true;
           if (lane == 0) {
-            bulk_wait0();  // this warp's reductions have been performed
-            fence_proxy_async_global();
+            if (ld_acquire_gpu(sem) != turn) {
+              const uint64_t t0 = global_ns();
+              while (ld_acquire_gpu(sem) != turn) {
+                if (global_ns() - t0 > kWaitLimitNs) {
+                  record_error(DEV_ERR_TIMEOUT, BWD_SITE_SEM);
+                  mine = false;
+                  break;
+                }
+              }
+            }
+            fence_proxy_async_global();  // our reductions come after the acquire
           }
-        }
-        __syncwarp();
-        mbar_arrive(dq_done);
-        if (c == 0) {
-          if (mbar_wait(dq_done, st & 1, BWD_SITE_SEM) && ok) {
-            __threadfence();
-            st_release_gpu(sem, (uint32_t)j + 1);
+          mine = __shfl_sync(0xffffffffu, mine, 0);
+          if (mine) {
+            reduce_partial();
+            if (lane == 0) {
+              bulk_wait0();  // this warp's reductions have been performed
+              fence_proxy_async_global();
+            }
+          }
+          __syncwarp();
+          mbar_arrive(dq_done);
+          if (c == 0) {
+            if (mbar_wait(dq_done, g & 1, BWD_SITE_SEM) && mine) {
+              __threadfence();
+              st_release_gpu(sem, turn + 1);
+            }
           }
         }
       }
@@ -739,6 +881,7 @@ __global__ void __launch_bounds__(512, 1)
 
   tc_fence_before();
   __syncthreads();
+  BWD_TRACE(threadIdx.x == 0, 4001);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

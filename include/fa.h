@@ -92,8 +92,9 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
 /*
  * Bytes of device scratch that fa_bwd needs for these sizes: an fp32 dQ
  * accumulator [B, H, S, D], one 32-byte row per query (LSE and the row term
- * D_i = dO_i . O_i, as bf16 parts, rows padded to multiples of 128), and the
- * ordering counters of deterministic mode, each 256-byte aligned.
+ * D_i = dO_i . O_i, as bf16 parts, rows padded to multiples of 128), the
+ * ordering counters of deterministic mode and the work counter of the
+ * backward's persistent grid, each 256-byte aligned.
  * Returns 0 for unsupported sizes.
  * This is the first half of the two-phase call of the operator in
  * "ops-transformer里的FlashAttention", "ops-transformer里的完整算子": a size
@@ -157,8 +158,9 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
  * must run in this order on one stream):
  *   fa_bwd_preprocess  D_i = dO_i . O_i and LSE into the workspace (as
  *                      the per-query rows of an extra product step);
- *                      clears the dQ accumulator and the deterministic-mode
- *                      counters.
+ *                      clears the dQ accumulator, the deterministic-mode
+ *                      counters and the work counter fa_bwd_main claims
+ *                      its units from.
  *   fa_bwd_main        the tiled pass over key/value tiles: writes dk, dv
  *                      and accumulates unscaled dQ (fp32) in the workspace.
  *   fa_bwd_finish      dq = scale * accumulated dQ, rounded to the dtype.
