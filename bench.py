@@ -133,6 +133,75 @@ def cpu_cores():
 
 # ------------------------------------------------------------------ clocks
 
+class NvmlClockSampler:
+    """SM clock, power and clock-event reasons read through NVML (read-only
+    queries) by a background thread, about once per millisecond, so that even
+    a timed region of a few milliseconds gets many samples.  Rows carry a
+    time.time() stamp like the nvidia-smi sampler's."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, uuid: str | None, index: int):
+        import threading
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        self.h = (pynvml.nvmlDeviceGetHandleByUUID(uuid) if uuid else pynvml.nvmlDeviceGetHandleByIndex(index))
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.bits = [(name, getattr(pynvml, attr)) for name, attr in self.REASONS]
+        self.rows, self.stop_evt = [], threading.Event()
+        self.t0 = self.t1 = None
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_evt.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                power = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+            except Exception:
+                break
+            self.rows.append(dict(ts=time.time(), sm=sm, sm_max=self.max_mhz, power=power,
+                                  reasons=[n for n, b in self.bits if reasons & b]))
+            self.stop_evt.wait(0.001)
+
+    def stop(self):
+        self.stop_evt.set()
+        self.thread.join(timeout=5)
+        try:
+            self.nv.nvmlShutdown()
+        except Exception:
+            pass
+        return self.rows
+
+    def summary(self, rows, t0=None, t1=None):
+        return clock_summary(rows, self.t0 if t0 is None else t0, self.t1 if t1 is None else t1, "nvml")
+
+
+def clock_summary(rows, t0, t1, source):
+    """Median SM clock, reasons and sample counts of the rows inside [t0, t1]
+    (all rows when none falls inside)."""
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": source}
+    inside = [r for r in rows if t0 is not None and t0 <= r["ts"] <= t1]
+    use = inside or rows
+    reasons = sorted({n for r in use for n in r["reasons"]})
+    return {"sm_mhz": statistics.median(r["sm"] for r in use), "sm_max_mhz": max(r["sm_max"] for r in use),
+            "reasons": reasons, "samples": len(use), "samples_in_timed_region": len(inside),
+            "power_w_max": max((r["power"] or 0.0) for r in use), "source": source}
+
+
+def start_clock_sampler(gpu_uuid, index):
+    try:
+        return NvmlClockSampler(gpu_uuid, index)
+    except Exception:
+        return ClockSampler(gpu_uuid)
+
+
 class ClockSampler:
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -173,15 +242,10 @@ class ClockSampler:
                 continue
         return rows
 
-    def summary(self, rows):
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        inside = [r for r in rows if self.t0 is not None and self.t0 - 0.15 <= r["ts"] <= self.t1 + 0.15]
-        use = inside or rows
-        reasons = sorted({n for r in use for n in r["reasons"]})
-        return {"sm_mhz": statistics.median(r["sm"] for r in use), "sm_max_mhz": max(r["sm_max"] for r in use),
-                "reasons": reasons, "samples": len(use), "samples_in_timed_region": len(inside),
-                "power_w_max": max((r["power"] or 0.0) for r in use)}
+    def summary(self, rows, t0=None, t1=None):
+        t0 = self.t0 if t0 is None else t0
+        t1 = self.t1 if t1 is None else t1
+        return clock_summary(rows, None if t0 is None else t0 - 0.15, None if t1 is None else t1 + 0.15, "nvidia-smi")
 
 
 # ------------------------------------------------------------------ CPU oracle legs
@@ -388,7 +452,7 @@ def main():
         gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         pass
-    sampler = ClockSampler(gpu_id)
+    sampler = start_clock_sampler(gpu_id, local)
     time.sleep(0.3)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     barrier()
@@ -402,8 +466,24 @@ def main():
     barrier()
     sampler.t1 = time.time()
     launches = fa.fa_launch_count() - launches0
+    fa.check_device_error()
+
+    # ---- sustained: the same step back to back (no flush in between) for
+    # about two seconds, clocks sampled over the whole run
+    sus_n = max(1, int(2.0 / max(1e-4, statistics.mean(e[0].elapsed_time(e[4]) for e in evs) * 1e-3)))
+    sus_e0, sus_e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    sus_t0 = time.time()
+    sus_e0.record(stream)
+    for _ in range(sus_n):
+        step()
+    sus_e1.record(stream)
+    torch.cuda.synchronize()
+    sus_t1 = time.time()
     clock_rows = sampler.stop()
     fa.check_device_error()
+    sus_ms = max_over_ranks({"s": sus_e0.elapsed_time(sus_e1) / sus_n}, device=dev)["s"]
 
     t_fwd = [e[0].elapsed_time(e[1]) for e in evs]
     t_pre = [e[1].elapsed_time(e[2]) for e in evs]
@@ -516,6 +596,11 @@ def main():
         decode["roofline"].update(achieved=d_gbs, frac=d_gbs / pk["hbm_gbs"])
 
     clocks = sampler.summary(clock_rows)
+    sus_clocks = sampler.summary(clock_rows, sus_t0, sus_t1)
+    sustained = {"steps": sus_n, "ms_per_step": sus_ms, "value": job_tflops(world, f_fwd + f_bwd, sus_ms),
+                 "unit": "TFLOP/s", "l2": "not flushed (steps back to back)", "clocks": sus_clocks,
+                 "ms_x_sm_mhz": sus_ms * (sus_clocks["sm_mhz"] or 0.0)}
+    clocks["ms_x_sm_mhz"] = ms["step"] * (clocks["sm_mhz"] or 0.0)
     if rank == 0:
         out = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -529,7 +614,7 @@ def main():
             "fwd_bwd_pct_of_2250": 100 * fb_tf / DATASHEET_TFLOPS,
             "fwd_frac_of_measured": fwd_tf / pk["bf16_tflops"], "bwd_frac_of_measured": bwd_tf / pk["bf16_tflops"],
             "kernel_ms": ms, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches, "clocks": clocks, "decode": decode,
+            "gpu_launches": launches, "clocks": clocks, "sustained": sustained, "decode": decode,
         }
         print(json.dumps(out), flush=True)
     if world > 1:

@@ -78,7 +78,7 @@
 // Timeline hooks: BWD_TRACE(condition, slot) records a clock at a point of
 // the pipeline in builds that define it; it compiles to nothing otherwise.
 #ifndef BWD_TRACE
-#define BWD_TRACE(cond, slot) ((void)0)
+#define BWD_TRACE(cond, slot) ((void)sizeof((cond) ? 1 : 0))
 #endif
 
 namespace fa {
