@@ -382,9 +382,16 @@ void* noalloc_scratch() {
 struct DecWs {
   size_t lse, total;
 };
+// Balanced mode runs at most this many CTAs (one per SM, B200 has 148).
+constexpr int kDecGridMax = 1024;
+
+// Partial results: rows * n_splits of them, or in balanced mode (n_splits =
+// 0) one per (cache, CTA) slot and query head of its group: at most
+// (B * Hkv + grid) * group <= B * Hq + kDecGridMax * 16 (group <= 16).
 DecWs dec_layout(long long rows, int n_splits, int D) {  // rows = B * Hq
-  const size_t o_bytes = up256((size_t)rows * n_splits * D * 4);
-  return {o_bytes, o_bytes + up256((size_t)rows * n_splits * 4)};
+  const long long parts = n_splits > 0 ? rows * n_splits : rows + (long long)kDecGridMax * 16;
+  const size_t o_bytes = up256((size_t)parts * D * 4);
+  return {o_bytes, o_bytes + up256((size_t)parts * 4)};
 }
 
 // Split count for B * Hkv cache streams of up to L_max keys: the fewest
@@ -419,29 +426,38 @@ fa_status launch_decode_t(const fa::DecParams& p, cudaStream_t st) {
     return FA_ERR_CUDA;
   if (set_smem<fa::decode_split_kernel<D, BF16>>(C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
   cudaError_t e;
-  const long long ctas = (long long)p.n_splits * p.Hkv * p.B;
-  if (p.n_splits >= 2 && p.n_splits <= kDecClusterMax && ctas <= sm_count()) {
-    // the splits of one (sequence, KV head) as one cluster, merged in-kernel
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.n_splits, p.Hkv, p.B);
-    cfg.blockDim = dim3(128);
-    cfg.dynamicSmemBytes = C::SMEM;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p.n_splits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, fa::decode_split_kernel<D, BF16>, mk, mv, p);
+  if (p.n_splits == 0) {
+    // balanced mode: the caches' tiles over one CTA per SM, then the merge
+    if (set_smem<fa::decode_balanced_kernel<D, BF16>>(C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
+    fa::decode_balanced_kernel<D, BF16><<<(unsigned)p.grid, 128, C::SMEM, st>>>(mk, mv, p);
     g_launches.fetch_add(1);
-    return from_cuda(e);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return from_cuda(e);
+  } else {
+    const long long ctas = (long long)p.n_splits * p.Hkv * p.B;
+    if (p.n_splits >= 2 && p.n_splits <= kDecClusterMax && ctas <= sm_count()) {
+      // the splits of one (sequence, KV head) as one cluster, merged in-kernel
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(p.n_splits, p.Hkv, p.B);
+      cfg.blockDim = dim3(128);
+      cfg.dynamicSmemBytes = C::SMEM;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = p.n_splits;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      e = cudaLaunchKernelEx(&cfg, fa::decode_split_kernel<D, BF16>, mk, mv, p);
+      g_launches.fetch_add(1);
+      return from_cuda(e);
+    }
+    fa::decode_split_kernel<D, BF16><<<dim3(p.n_splits, p.Hkv, p.B), 128, C::SMEM, st>>>(mk, mv, p);
+    g_launches.fetch_add(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.n_splits == 1) return from_cuda(e);  // one split writes O and LSE itself
   }
-  fa::decode_split_kernel<D, BF16><<<dim3(p.n_splits, p.Hkv, p.B), 128, C::SMEM, st>>>(mk, mv, p);
-  g_launches.fetch_add(1);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || p.n_splits == 1) return from_cuda(e);  // one split writes O and LSE itself
   // the merge as a programmatic dependent launch: it is scheduled while the
   // split kernel runs and waits (griddepcontrol.wait) for its results
   cudaLaunchConfig_t cfg = {};
@@ -664,7 +680,7 @@ int fa_decode_num_splits(int B, int Hkv, int L_max) {
 }
 
 size_t fa_decode_workspace_size(int B, int Hq, int n_splits, int D) {
-  if (B <= 0 || Hq <= 0 || n_splits <= 0 || (D != 64 && D != 128)) return 0;
+  if (B <= 0 || Hq <= 0 || n_splits < 0 || n_splits > 1024 || (D != 64 && D != 128)) return 0;
   return dec_layout((long long)B * Hq, n_splits, D).total;
 }
 
@@ -678,7 +694,7 @@ fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, con
   if (B == 0 || Hq == 0) return FA_OK;
   if (Hkv == 0 || Hq % Hkv) return FA_ERR_INVALID_ARG;
   if (Hq / Hkv > 16) return FA_ERR_UNSUPPORTED;
-  if (n_splits < 1 || n_splits > 1024) return FA_ERR_INVALID_ARG;
+  if (n_splits < 0 || n_splits > 1024) return FA_ERR_INVALID_ARG;
   if (B > 65535 || Hkv > 65535 || (long long)B * Hq > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   if (!ptrs_ok({q, k_cache, v_cache, o, lse}) || !seq_lens || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
     return FA_ERR_INVALID_ARG;
@@ -695,6 +711,9 @@ fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, con
   p.o = o;
   p.lse = lse;
   p.B = B, p.Hq = Hq, p.Hkv = Hkv, p.L = L_max, p.n_splits = n_splits, p.group = Hq / Hkv;
+  p.tpp = std::max(1, (L_max + fa::DecCfg<64>::KT - 1) / fa::DecCfg<64>::KT);
+  p.tiles = (long long)B * Hkv * p.tpp;
+  p.grid = (int)std::min<long long>(std::min(sm_count(), kDecGridMax), p.tiles);
   p.scale_log2 = scale * 1.4426950408889634f;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (D == 128) return dt == FA_BF16 ? launch_decode_t<128, true>(p, st) : launch_decode_t<128, false>(p, st);

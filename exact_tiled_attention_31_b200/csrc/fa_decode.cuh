@@ -42,12 +42,18 @@ struct DecParams {
   const uint16_t* k;     // [B, Hkv, L, D]
   const uint16_t* v;     // [B, Hkv, L, D]
   const int* seq_lens;   // [B] valid cached keys per sequence
-  float* o_part;         // [B, Hq, n_splits, D] fp32, normalised over the split's keys
-  float* lse_part;       // [B, Hq, n_splits] natural log, -inf for an empty split
+  float* o_part;         // fp32 partial O, normalised over its keys: [B, Hq, n_splits, D]
+                         // (balanced mode: [B * Hkv + grid, group, D], see decode_balanced_kernel)
+  float* lse_part;       // natural log, -inf for an empty key range: [B, Hq, n_splits]
+                         // (balanced mode: [B * Hkv + grid, group])
   void* o;               // [B, Hq, D] 16-bit output
   float* lse;            // [B, Hq]
   int B, Hq, Hkv, L, n_splits, group;
   float scale_log2;      // scale * log2(e)
+  // balanced mode (n_splits = 0): the B * Hkv caches' 32-key tiles, tpp per
+  // cache, are dealt out evenly over `grid` CTAs
+  long long tiles;
+  int tpp, grid;
 };
 
 template <int D>
@@ -141,34 +147,27 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
   }
 }
 
+// This thread's share of one CTA's result over a key range: the (max, sum
+// of exponentials, sum of rounded exponentials, 16 columns of unnormalised O)
+// of query row `row` (a query head of the group) and columns [16 part, +16).
+struct DecPart {
+  float mm, lt, lrt, acc[16];
+  int row, part;
+  bool active;
+};
+
+// The CTA's four warps over keys [start, end) of cache (b, kvh), then merged
+// across the warps through shared memory.  `it` counts the tiles this warp
+// has taken from its ring so far (it carries the barrier phases from one
+// range to the next); every thread of the CTA calls this with the same range.
 template <int D, bool BF16>
-__global__ void __launch_bounds__(128, 1)
-    decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                        const DecParams p) {
+__device__ __forceinline__ void dec_range(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const DecParams& p,
+                                          uint8_t* dsm, uint64_t (*bars)[DecCfg<D>::STAGES], int b, int kvh,
+                                          int start, int end, uint32_t& it, DecPart& out) {
   using C = DecCfg<D>;
-  extern __shared__ uint8_t dsm_raw[];
-  __shared__ uint64_t bars[C::WARPS][C::STAGES];
-  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int len = min(max(p.seq_lens[b], 0), p.L);
-  // this split's keys: [start, end), a multiple of KT long except at the end
-  const int per = ((len + p.n_splits - 1) / p.n_splits + C::KT - 1) / C::KT * C::KT;
-  const int start = split * per, end = min(len, start + per);
   const int n_tiles = end > start ? (end - start + C::KT - 1) / C::KT : 0;
   const int bh = b * p.Hkv + kvh;  // cache head index (third tensor-map coordinate)
-  if (lane == 0) {
-    for (int s = 0; s < C::STAGES; ++s) mbar_init(&bars[warp][s], 1);
-    fence_mbar_init();
-  }
-  if (threadIdx.x == 0) {
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-  }
-  // the merge launch may start once every block has got here; it still waits
-  // for this grid's completion before reading the partial results
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __syncwarp();
 
   // Q as the A operand (rows = the group's query heads, padded to 16 with zeros)
   const int r0 = lane >> 2, r1 = r0 + 8, cq = 2 * (lane & 3);
@@ -188,15 +187,15 @@ __global__ void __launch_bounds__(128, 1)
   uint8_t* vbuf = kbuf + C::STAGES * C::TILE;
   const uint16_t* kh = p.k + (size_t)bh * p.L * D;
   const uint16_t* vh = p.v + (size_t)bh * p.L * D;
-  // The warp's i-th tile is tile warp + WARPS * i of the split, in stage
-  // i % STAGES.  A whole tile comes by TMA; the one tile that runs past
-  // `end` (always the split's last, so the warp's last) by cp.async with
-  // the rows past `end` zero-filled.
+  // The warp's i-th tile of the range is tile warp + WARPS * i, in stage
+  // (it + i) % STAGES.  A whole tile comes by TMA; the one tile that runs past
+  // `end` (always the range's last, so the warp's last) by cp.async with the
+  // rows past `end` zero-filled.
   auto full_tile = [&](int i) { return start + C::KT * (warp + C::WARPS * i) + C::KT <= end; };
   auto issue = [&](int i) {
     const int t = warp + C::WARPS * i;
     if (t >= n_tiles) return;
-    const int key0 = start + C::KT * t, s = i % C::STAGES;
+    const int key0 = start + C::KT * t, s = (it + i) % C::STAGES;
     uint8_t* kd = kbuf + s * C::TILE;
     uint8_t* vd = vbuf + s * C::TILE;
     if (key0 + C::KT <= end) {
@@ -234,18 +233,24 @@ __global__ void __launch_bounds__(128, 1)
   for (int i = 0; i < C::STAGES - 1; ++i) issue(i);
   for (int i = 0; i < my_tiles; ++i) {
     issue(i + C::STAGES - 1);
-    const int t = warp + C::WARPS * i, st = i % C::STAGES;
+    const int t = warp + C::WARPS * i, st = (it + i) % C::STAGES;
     if (full_tile(i)) {
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[warp][st], (i / C::STAGES) & 1, DEC_SITE_KV));
+      const bool ok =
+          __all_sync(0xffffffffu, mbar_wait(&bars[warp][st], ((it + i) / C::STAGES) & 1, DEC_SITE_KV));
       if (!ok) {  // error recorded: let the warp's copies in flight, this tile's included, land
                   // (bounded waits again), then stop
         for (int j = i; j < min(i + C::STAGES, my_tiles); ++j)
-          if (full_tile(j)) mbar_wait(&bars[warp][j % C::STAGES], (j / C::STAGES) & 1, DEC_SITE_DRAIN);
+          if (full_tile(j))
+            mbar_wait(&bars[warp][(it + j) % C::STAGES], ((it + j) / C::STAGES) & 1, DEC_SITE_DRAIN);
         break;
       }
     } else {
       cp_async_wait<0>();
       __syncwarp();
+      // a copied tile completes its stage's barrier phase too, so that every
+      // tile, however it came, moves its stage on by exactly one phase (the
+      // next range of a balanced-mode CTA relies on the parities)
+      if (lane == 0) mbar_arrive(&bars[warp][st]);
     }
     const uint32_t ks = smem_addr(kbuf + st * C::TILE), vs = smem_addr(vbuf + st * C::TILE);
     // S = Q K^T: 16 rows x 32 keys (4 tiles of 8)
@@ -322,6 +327,7 @@ __global__ void __launch_bounds__(128, 1)
     __syncwarp();  // every lane is done with this stage before it is refilled
   }
   cp_async_wait<0>();
+  it += (uint32_t)my_tiles;
 
   // the lane's shares of the row sums -> the row's (4 lanes of a quad)
 #pragma unroll
@@ -352,25 +358,74 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   // thread -> (row, 16 of the D columns): this CTA's (max, sums, unnormalised O)
   constexpr int PARTS = D / 16;
-  const int row = threadIdx.x / PARTS, part = threadIdx.x % PARTS;
-  const bool active = row < p.group && threadIdx.x < 16 * PARTS;
-  float mm = -INFINITY, lt = 0.f, lrt = 0.f, acc[16];
+  out.row = threadIdx.x / PARTS;
+  out.part = threadIdx.x % PARTS;
+  out.active = out.row < p.group && threadIdx.x < 16 * PARTS;
+  out.mm = -INFINITY;
+  out.lt = out.lrt = 0.f;
 #pragma unroll
-  for (int d = 0; d < 16; ++d) acc[d] = 0.f;
-  if (active) {
+  for (int d = 0; d < 16; ++d) out.acc[d] = 0.f;
+  if (out.active) {
     const float* w0 = reinterpret_cast<const float*>(dsm);
 #pragma unroll
-    for (int w = 0; w < C::WARPS; ++w) mm = fmaxf(mm, w0[w * C::SCRATCH + row]);
+    for (int w = 0; w < C::WARPS; ++w) out.mm = fmaxf(out.mm, w0[w * C::SCRATCH + out.row]);
 #pragma unroll
     for (int w = 0; w < C::WARPS; ++w) {
       const float* wp = w0 + w * C::SCRATCH;
-      const float sc = mm == -INFINITY ? 0.f : ex2(wp[row] - mm);  // empty warp ranges weigh 0
-      lt += wp[16 + row] * sc;
-      lrt += wp[32 + row] * sc;
+      const float sc = out.mm == -INFINITY ? 0.f : ex2(wp[out.row] - out.mm);  // empty warp ranges weigh 0
+      out.lt += wp[16 + out.row] * sc;
+      out.lrt += wp[32 + out.row] * sc;
 #pragma unroll
-      for (int d = 0; d < 16; ++d) acc[d] += wp[48 + row * D + 16 * part + d] * sc;
+      for (int d = 0; d < 16; ++d) out.acc[d] += wp[48 + out.row * D + 16 * out.part + d] * sc;
     }
   }
+}
+
+// A CTA's normalised partial O (fp32) and its LSE for one key range.
+template <int D>
+__device__ __forceinline__ void dec_store_part(const DecPart& r, float* o_part_row, float* lse_part_row) {
+  const float inv = r.lrt > 0.f ? 1.f / r.lrt : 0.f;
+  float4* dst = reinterpret_cast<float4*>(o_part_row + 16 * r.part);
+#pragma unroll
+  for (int d = 0; d < 4; ++d)
+    dst[d] = make_float4(r.acc[4 * d] * inv, r.acc[4 * d + 1] * inv, r.acc[4 * d + 2] * inv, r.acc[4 * d + 3] * inv);
+  if (r.part == 0) *lse_part_row = r.lt > 0.f ? (r.mm + __log2f(r.lt)) * 0.69314718055994531f : -INFINITY;
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(128, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        const DecParams p) {
+  using C = DecCfg<D>;
+  extern __shared__ uint8_t dsm_raw[];
+  __shared__ uint64_t bars[C::WARPS][C::STAGES];
+  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int len = min(max(p.seq_lens[b], 0), p.L);
+  // this split's keys: [start, end), a multiple of KT long except at the end
+  const int per = ((len + p.n_splits - 1) / p.n_splits + C::KT - 1) / C::KT * C::KT;
+  const int start = split * per, end = min(len, start + per);
+  if (lane == 0) {
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(&bars[warp][s], 1);
+    fence_mbar_init();
+  }
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  // the merge launch may start once every block has got here; it still waits
+  // for this grid's completion before reading the partial results
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __syncwarp();
+
+  uint32_t it = 0;
+  DecPart r;
+  dec_range<D, BF16>(tm_k, tm_v, p, dsm, bars, b, kvh, start, end, it, r);
+  const int row = r.row, part = r.part;
+  const bool active = r.active;
+  const float mm = r.mm, lt = r.lt, lrt = r.lrt;
+  const float* acc = r.acc;
   const size_t qrow = (size_t)b * p.Hq + kvh * p.group + row;
 
   if (cluster_nctarank() > 1) {
@@ -391,16 +446,16 @@ __global__ void __launch_bounds__(128, 1)
     if (cluster_ctarank() == 0 && active) {
       const uint32_t nct = cluster_nctarank();
       float M = -INFINITY;
-      for (uint32_t r = 0; r < nct; ++r) M = fmaxf(M, ld_dsmem(dsmem_addr(pub + row, r)));
+      for (uint32_t q = 0; q < nct; ++q) M = fmaxf(M, ld_dsmem(dsmem_addr(pub + row, q)));
       float L = 0.f, LR = 0.f, O[16];
 #pragma unroll
       for (int d = 0; d < 16; ++d) O[d] = 0.f;
-      for (uint32_t r = 0; r < nct; ++r) {
-        const float mr = ld_dsmem(dsmem_addr(pub + row, r));
+      for (uint32_t q = 0; q < nct; ++q) {
+        const float mr = ld_dsmem(dsmem_addr(pub + row, q));
         const float w = M == -INFINITY ? 0.f : ex2(mr - M);
-        L += w * ld_dsmem(dsmem_addr(pub + 16 + row, r));
-        LR += w * ld_dsmem(dsmem_addr(pub + 32 + row, r));
-        const uint32_t oa = dsmem_addr(pub + 48 + row * D + 16 * part, r);
+        L += w * ld_dsmem(dsmem_addr(pub + 16 + row, q));
+        LR += w * ld_dsmem(dsmem_addr(pub + 32 + row, q));
+        const uint32_t oa = dsmem_addr(pub + 48 + row * D + 16 * part, q);
 #pragma unroll
         for (int d = 0; d < 4; ++d) {
           const float4 v = ld_dsmem4(oa + 16 * d);
@@ -425,9 +480,8 @@ __global__ void __launch_bounds__(128, 1)
   }
 
   if (active) {
-    const float inv = lrt > 0.f ? 1.f / lrt : 0.f;
-    const float lse = lt > 0.f ? (mm + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
     if (p.n_splits == 1) {  // the split is the whole cache: final O and LSE
+      const float inv = lrt > 0.f ? 1.f / lrt : 0.f;
       uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + qrow * D + 16 * part);
 #pragma unroll
       for (int d = 0; d < 2; ++d)
@@ -435,34 +489,102 @@ __global__ void __launch_bounds__(128, 1)
                             pack2<BF16>(acc[8 * d + 2] * inv, acc[8 * d + 3] * inv),
                             pack2<BF16>(acc[8 * d + 4] * inv, acc[8 * d + 5] * inv),
                             pack2<BF16>(acc[8 * d + 6] * inv, acc[8 * d + 7] * inv));
-      if (part == 0) p.lse[qrow] = lse;
+      if (part == 0) p.lse[qrow] = lt > 0.f ? (mm + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
     } else {  // partial result for decode_merge_kernel
       const size_t orow = qrow * p.n_splits + split;
-      float4* dst = reinterpret_cast<float4*>(p.o_part + orow * D + 16 * part);
-#pragma unroll
-      for (int d = 0; d < 4; ++d)
-        dst[d] = make_float4(acc[4 * d] * inv, acc[4 * d + 1] * inv, acc[4 * d + 2] * inv, acc[4 * d + 3] * inv);
-      if (part == 0) p.lse_part[orow] = lse;
+      dec_store_part<D>(r, p.o_part + orow * D, p.lse_part + orow);
     }
   }
 }
 
-// O and LSE of each (sequence, query head) from its splits: LSE = log sum
+// Balanced mode: the caches' 32-key tiles, in (sequence, KV head) order,
+// are dealt out in equal contiguous runs to `grid` CTAs (one per SM), so every
+// SM streams the same number of cache bytes whatever the batch and lengths.
+// A run can cover the end of one cache and the start of the next: the CTA
+// writes one partial result per cache it meets.  Cache pr's part from CTA c
+// goes to slot pr + c: along the tile list both only grow, and every new
+// part moves to a new cache, a new CTA or both, so slots never collide and
+// B * Hkv + grid of them are enough.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(128, 1)
+    decode_balanced_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                           const DecParams p) {
+  using C = DecCfg<D>;
+  extern __shared__ uint8_t dsm_raw[];
+  __shared__ uint64_t bars[C::WARPS][C::STAGES];
+  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(&bars[warp][s], 1);
+    fence_mbar_init();
+  }
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __syncwarp();
+  const long long c = blockIdx.x;
+  const long long t0 = c * p.tiles / p.grid, t1 = (c + 1) * p.tiles / p.grid;  // this CTA's tiles [t0, t1)
+  uint32_t it = 0;
+  if (t1 <= t0) return;
+  const long long first_pair = t0 / p.tpp, last_pair = (t1 - 1) / p.tpp;  // the caches this run meets
+  for (long long pr = first_pair; pr <= last_pair; ++pr) {
+    const int b = (int)(pr / p.Hkv), kvh = (int)(pr - (long long)b * p.Hkv);
+    const int len = min(max(p.seq_lens[b], 0), p.L);
+    const long long a0 = max(t0, pr * p.tpp) - pr * p.tpp, a1 = min(t1, (pr + 1) * p.tpp) - pr * p.tpp;
+    const int start = min((int)a0 * C::KT, len), end = min((int)a1 * C::KT, len);
+    DecPart r;
+    dec_range<D, BF16>(tm_k, tm_v, p, dsm, bars, b, kvh, start, end, it, r);
+    if (r.active) {
+      const size_t slot = (size_t)(pr + c) * p.group + r.row;
+      dec_store_part<D>(r, p.o_part + slot * D, p.lse_part + slot);
+    }
+    __syncthreads();  // the scratch in the tile buffers is read before the next range refills them
+  }
+}
+
+// O and LSE of each (sequence, query head) from its parts: LSE = log sum
 // exp(LSE_s), O = sum exp(LSE_s - LSE) O_s.  One block of D threads per row.
-// Launched as a programmatic dependent of decode_split_kernel: its blocks may
-// be resident before the split kernel ends and wait here for its results.
+// Launched as a programmatic dependent of the split or balanced kernel: its
+// blocks may be resident before that kernel ends and wait here for its
+// results.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(D) decode_merge_kernel(const DecParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const size_t row = blockIdx.x;  // b * Hq + h
-  const float* lp = p.lse_part + row * p.n_splits;
+  // the row's parts: n of them, part s at index part_at(s) of lse_part (and
+  // of o_part in rows of D)
+  int n;
+  size_t first, rest0, rest_stride;  // part 0 at `first`, part s >= 1 at rest0 + (s - 1) * rest_stride
+  if (p.n_splits > 0) {
+    n = p.n_splits;
+    first = row * p.n_splits;
+    rest0 = first + 1;
+    rest_stride = 1;
+  } else {
+    // balanced mode: the cache's tiles [pr tpp, (pr + 1) tpp) were run by CTAs
+    // c0 .. c1, whose parts sit in slots pr + c0 .. pr + c1
+    const long long b = (long long)(row / p.Hq), h = (long long)(row % p.Hq);
+    const long long pr = b * p.Hkv + h / p.group;
+    const size_t gi = (size_t)(h % p.group);
+    // CTA whose run holds tile x: the largest c with floor(c tiles / grid) <= x
+    auto cta_of = [&](long long x) { return ((x + 1) * p.grid - 1) / p.tiles; };
+    const long long c0 = cta_of(pr * p.tpp), c1 = cta_of((pr + 1) * p.tpp - 1);
+    n = (int)(c1 - c0 + 1);
+    first = (size_t)(pr + c0) * p.group + gi;
+    rest0 = first + p.group;
+    rest_stride = p.group;
+  }
+  auto part_at = [&](int s) { return s == 0 ? first : rest0 + (size_t)(s - 1) * rest_stride; };
   float mx = -INFINITY;
-  for (int s = 0; s < p.n_splits; ++s) mx = fmaxf(mx, lp[s]);
+  for (int s = 0; s < n; ++s) mx = fmaxf(mx, p.lse_part[part_at(s)]);
   float tot = 0.f, acc = 0.f;
-  for (int s = 0; s < p.n_splits; ++s) {
-    const float w = mx == -INFINITY ? 0.f : __expf(lp[s] - mx);
+  for (int s = 0; s < n; ++s) {
+    const size_t idx = part_at(s);
+    const float w = mx == -INFINITY ? 0.f : __expf(p.lse_part[idx] - mx);
     tot += w;
-    acc += w * p.o_part[(row * p.n_splits + s) * D + threadIdx.x];
+    acc += w * p.o_part[idx * D + threadIdx.x];
   }
   const float o = tot > 0.f ? acc / tot : 0.f;
   uint16_t* dst = static_cast<uint16_t*>(p.o) + row * D + threadIdx.x;

@@ -130,7 +130,12 @@ def test_decode_workspace_splits_and_argument_errors(lib):
     for B, Hq, n, D in [(8, 32, 16, 128), (3, 5, 7, 64), (1, 1, 1, 128)]:
         assert fa.fa_decode_workspace_size(B, Hq, n, D) == up(B * Hq * n * D * 4) + up(B * Hq * n * 4)
     assert fa.fa_decode_workspace_size(1, 1, 1, 96) == 0
-    assert fa.fa_decode_workspace_size(1, 1, 0, 64) == 0
+    assert fa.fa_decode_workspace_size(1, 1, -1, 64) == 0
+    # balanced mode (n_splits = 0): one part per (cache, CTA) slot and query head,
+    # at most B * Hq + 1024 CTAs x 16 heads of a group
+    for B, Hq, D in [(8, 32, 128), (1, 1, 64)]:
+        rows = B * Hq + 1024 * 16
+        assert fa.fa_decode_workspace_size(B, Hq, 0, D) == up(rows * D * 4) + up(rows * 4)
     # the library's split choice: 1..64, at least 256 keys per split
     for B, Hkv, L in [(8, 8, 8192), (1, 1, 100), (1, 8, 32768), (64, 8, 2048), (1, 1, 1 << 20)]:
         n = fa.fa_decode_num_splits(B, Hkv, L)
@@ -148,8 +153,9 @@ def test_decode_workspace_splits_and_argument_errors(lib):
     assert call(Hkv=0) == fa.api.FA_ERR_INVALID_ARG
     assert call(Hq=34, Hkv=2, wsb=1 << 30) == fa.api.FA_ERR_UNSUPPORTED   # group of 17 query heads
     assert call(D=96) == fa.api.FA_ERR_UNSUPPORTED
-    assert call(n=0) == fa.api.FA_ERR_INVALID_ARG
+    assert call(n=-1) == fa.api.FA_ERR_INVALID_ARG
     assert call(n=1025) == fa.api.FA_ERR_INVALID_ARG
+    assert call(n=0, wsb=fa.fa_decode_workspace_size(2, 8, 0, 64) - 1) == fa.api.FA_ERR_INVALID_ARG
     assert call(lens=A + 2) == fa.api.FA_ERR_INVALID_ARG      # misaligned seq_lens
     assert call(q=A + 8) == fa.api.FA_ERR_INVALID_ARG         # misaligned q
     assert call(ws=A + 64) == fa.api.FA_ERR_INVALID_ARG       # workspace not 256-byte aligned

@@ -128,3 +128,52 @@ def test_decode_full_size_sampled(cuda_device):
     ro, rl = _ref(t, 1.0 / math.sqrt(128), [0, 7])
     check_o(o[[0, 7]], ro, "full size")
     check_lse(lse[[0, 7]], rl, "full size LSE")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,D,dtype", [
+    (4, 32, 8, 1000, 128, "bf16"),   # caches of 32 tiles over 128 CTAs: one cache per several CTAs
+    (40, 8, 4, 600, 128, "bf16"),    # 160 caches of 19 tiles over 148 CTAs: runs that span two caches
+    (3, 16, 1, 700, 64, "fp16"),     # multi-query, group 16, D = 64
+    (2, 10, 2, 33, 128, "fp16"),     # two tiles per cache, group 5 (padded rows): fewer tiles than SMs
+])
+def test_decode_balanced_matches_oracle(cuda_device, B, Hq, Hkv, L, D, dtype):
+    """Balanced mode (n_splits = 0): the caches' 32-key tiles dealt out evenly
+    over one CTA per SM, each cache's parts merged by their LSE."""
+    t = inputs.make_decode(B, Hq, Hkv, L, D, dtype, seed=B * L + D)
+    o, lse = _run(t, cuda_device, n_splits=0)
+    ro, rl = _ref(t, 1.0 / math.sqrt(D))
+    check_o(o, ro, f"balanced B{B} Hq{Hq} Hkv{Hkv} L{L} D{D} {dtype}")
+    check_lse(lse, rl, "balanced LSE")
+
+
+def test_decode_balanced_ragged_and_poisoned(cuda_device):
+    """Balanced mode over ragged lengths (empty, single key, tile edges, past
+    the cache) with every cache row at or past a length set to NaN."""
+    L, D = 300, 128
+    lens = [1, 31, 32, 33, 64, 65, 255, 299, 300, 1000, 0, 7]
+    t = inputs.make_decode(len(lens), 8, 2, L, D, "bf16", seed=6)
+    t["seq_lens"] = torch.tensor(lens, dtype=torch.int32)
+    clamped = [min(x, L) for x in lens]
+    live = [b for b, x in enumerate(lens) if x > 0]
+    ro, rl = _ref(dict(t, seq_lens=torch.tensor(clamped, dtype=torch.int32)), 0.1, live)
+    for b, n in enumerate(clamped):
+        t["k"][b, :, n:] = float("nan")
+        t["v"][b, :, n:] = float("nan")
+    o, lse = _run(t, cuda_device, n_splits=0, scale=0.1)
+    check_o(o[live], ro, "balanced ragged")
+    check_lse(lse[live], rl, "balanced ragged LSE")
+    empty = lens.index(0)
+    assert torch.all(o[empty] == 0)
+    assert torch.all(torch.isneginf(lse[empty]))
+
+
+def test_decode_long_context_sampled(cuda_device):
+    """One sequence with a 32768-key cache (B1 Hq32 Hkv8 D128 bf16), the
+    library's choice of cut and balanced mode, checked against the oracle."""
+    t = inputs.make_decode(1, 32, 8, 32768, 128, "bf16", seed=3)
+    t["seq_lens"] = torch.full((1,), 32768, dtype=torch.int32)
+    ro, rl = _ref(t, 1.0 / math.sqrt(128))
+    for n_splits in (None, 0):
+        o, lse = _run(t, cuda_device, n_splits=n_splits)
+        check_o(o, ro, f"long context, splits {n_splits}")
+        check_lse(lse, rl, "long context LSE")
