@@ -31,7 +31,8 @@ FA_BF16, FA_FP16 = 0, 1
 EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
            "fa_bwd_finish", "fa_bwd_noalloc", "fa_bwd_varlen_workspace_size", "fa_bwd_varlen", "fa_status_string",
            "fa_check_device_error", "fa_launch_count", "fa_selftest_timeout", "fa_decode_num_splits",
-           "fa_decode_workspace_size", "fa_decode", "fa_fwd_dropout", "fa_bwd_dropout")
+           "fa_decode_workspace_size", "fa_decode", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_varlen_dropout",
+           "fa_bwd_varlen_dropout")
 
 # Fixed scratch size of fa_bwd_noalloc (FA_BWD_NOALLOC_SCRATCH_BYTES in include/fa.h).
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -93,6 +94,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_fwd_dropout.restype = i
     lib.fa_bwd_dropout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, f, u64, u64, vp, sz, vp]
     lib.fa_bwd_dropout.restype = i
+    lib.fa_fwd_varlen_dropout.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, f, u64, u64, vp]
+    lib.fa_fwd_varlen_dropout.restype = i
+    lib.fa_bwd_varlen_dropout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, f, u64,
+                                          u64, vp, sz, vp]
+    lib.fa_bwd_varlen_dropout.restype = i
     lib.fa_launch_count.argtypes = []
     lib.fa_launch_count.restype = ctypes.c_uint64
     _lib = lib
@@ -161,6 +167,19 @@ def fa_bwd_dropout(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, causal, d
     return load_library().fa_bwd_dropout(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, int(causal), dt,
                                          int(deterministic), dropout_p, seed, offset, workspace, workspace_bytes,
                                          stream)
+
+
+def fa_fwd_varlen_dropout(q, k, v, o, lse, cu_seqlens, nseq, max_seqlen, total, H, D, scale, causal, dt, dropout_p,
+                          seed, offset, stream) -> int:
+    return load_library().fa_fwd_varlen_dropout(q, k, v, o, lse, cu_seqlens, nseq, max_seqlen, total, H, D, scale,
+                                                int(causal), dt, dropout_p, seed, offset, stream)
+
+
+def fa_bwd_varlen_dropout(q, k, v, o, dO, lse, dq, dk, dv, cu_seqlens, nseq, max_seqlen, total, H, D, scale, causal,
+                          dt, deterministic, dropout_p, seed, offset, workspace, workspace_bytes, stream) -> int:
+    return load_library().fa_bwd_varlen_dropout(q, k, v, o, dO, lse, dq, dk, dv, cu_seqlens, nseq, max_seqlen, total,
+                                                H, D, scale, int(causal), dt, int(deterministic), dropout_p, seed,
+                                                offset, workspace, workspace_bytes, stream)
 
 
 def fa_decode_num_splits(B, Hkv, L_max) -> int:
@@ -247,8 +266,10 @@ def forward(q, k, v, causal: bool, scale: float | None = None, out=None, lse=Non
 
 
 def forward_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool, scale: float | None = None,
-                   stream=None):
-    """Packed [H, T, D] forward; ``cu_seqlens`` is a device int32 tensor."""
+                   stream=None, dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
+    """Packed [H, T, D] forward; ``cu_seqlens`` is a device int32 tensor.
+    ``dropout_p`` > 0 drops P with sequence s taking the mask of batch index
+    s of a dense batch (fa_fwd_varlen_dropout)."""
     import torch
     H, T, D = q.shape
     _check((q, k, v), q.shape)
@@ -257,6 +278,13 @@ def forward_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool, scale: fl
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     o = torch.empty_like(q)
     lse = torch.empty((H, T), device=q.device, dtype=torch.float32)
+    if dropout_p:
+        st = fa_fwd_varlen_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                   cu_seqlens.data_ptr(), cu_seqlens.numel() - 1, int(max_seqlen), T, H, D, scale,
+                                   causal, _dt(q), float(dropout_p), int(seed), int(offset), _stream(stream))
+        if st != FA_OK:
+            raise FAError(st, "fa_fwd_varlen_dropout")
+        return o, lse
     st = fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                        cu_seqlens.data_ptr(), cu_seqlens.numel() - 1, int(max_seqlen), T, H, D, scale, causal,
                        _dt(q), _stream(stream))
@@ -299,8 +327,10 @@ def backward(q, k, v, o, do, lse, causal: bool, scale: float | None = None, dete
 
 
 def backward_varlen(q, k, v, o, do, lse, cu_seqlens, max_seqlen: int, causal: bool, scale: float | None = None,
-                    deterministic: bool = False, workspace=None, stream=None):
-    """dQ, dK, dV of a packed [H, T, D] batch given fa_fwd_varlen's O and LSE."""
+                    deterministic: bool = False, workspace=None, stream=None, dropout_p: float = 0.0, seed: int = 0,
+                    offset: int = 0):
+    """dQ, dK, dV of a packed [H, T, D] batch given fa_fwd_varlen's O and LSE
+    (with the forward's dropout_p, seed and offset, if it dropped)."""
     import torch
     H, T, D = q.shape
     _check((q, k, v, o, do), q.shape)
@@ -312,10 +342,16 @@ def backward_varlen(q, k, v, o, do, lse, cu_seqlens, max_seqlen: int, causal: bo
     nbytes = fa_bwd_varlen_workspace_size(nseq, int(max_seqlen), T, H, D)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(max(nbytes, 1), device=q.device, dtype=torch.uint8)
-    st = fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
-                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu_seqlens.data_ptr(), nseq, int(max_seqlen), T,
-                       H, D, scale, causal, _dt(q), deterministic, workspace.data_ptr(), workspace.numel(),
-                       _stream(stream))
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+            dk.data_ptr(), dv.data_ptr(), cu_seqlens.data_ptr(), nseq, int(max_seqlen), T, H, D, scale, causal, _dt(q),
+            deterministic)
+    if dropout_p:
+        st = fa_bwd_varlen_dropout(*args, float(dropout_p), int(seed), int(offset), workspace.data_ptr(),
+                                   workspace.numel(), _stream(stream))
+        if st != FA_OK:
+            raise FAError(st, "fa_bwd_varlen_dropout")
+        return dq, dk, dv
+    st = fa_bwd_varlen(*args, workspace.data_ptr(), workspace.numel(), _stream(stream))
     if st != FA_OK:
         raise FAError(st, "fa_bwd_varlen")
     return dq, dk, dv

@@ -128,9 +128,11 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 template <int D, bool BF16>
 fa_status dispatch_fwd(bool causal, bool varlen, bool dropout, const CUtensorMap& mq, const CUtensorMap& mk,
                        const CUtensorMap& mv, const fa::FwdParams& p, cudaStream_t st) {
-  if (dropout)  // dense batches only
-    return causal ? launch_fwd<D, BF16, true, false, true>(mq, mk, mv, p, st)
-                  : launch_fwd<D, BF16, false, false, true>(mq, mk, mv, p, st);
+  if (dropout)
+    return varlen ? (causal ? launch_fwd<D, BF16, true, true, true>(mq, mk, mv, p, st)
+                            : launch_fwd<D, BF16, false, true, true>(mq, mk, mv, p, st))
+                  : (causal ? launch_fwd<D, BF16, true, false, true>(mq, mk, mv, p, st)
+                            : launch_fwd<D, BF16, false, false, true>(mq, mk, mv, p, st));
   if (varlen)
     return causal ? launch_fwd<D, BF16, true, true>(mq, mk, mv, p, st)
                   : launch_fwd<D, BF16, false, true>(mq, mk, mv, p, st);
@@ -251,9 +253,11 @@ fa_status launch_bwd_main(const void* q, const void* k, const void* v, const voi
       !make_map_f32(&mdq, p.dq_acc, D, p.rows, p.heads) ||
       !make_map_cols(&mcols, p.cols, (long long)p.heads * p.nseq * p.S_pad))
     return FA_ERR_CUDA;
-  if (dropout)  // dense batches only
-    return causal ? launch_bwd_main_t<D, BF16, true, false, true>(mq, mk, mv, mdo, mdq, mcols, p, st)
-                  : launch_bwd_main_t<D, BF16, false, false, true>(mq, mk, mv, mdo, mdq, mcols, p, st);
+  if (dropout)
+    return varlen ? (causal ? launch_bwd_main_t<D, BF16, true, true, true>(mq, mk, mv, mdo, mdq, mcols, p, st)
+                            : launch_bwd_main_t<D, BF16, false, true, true>(mq, mk, mv, mdo, mdq, mcols, p, st))
+                  : (causal ? launch_bwd_main_t<D, BF16, true, false, true>(mq, mk, mv, mdo, mdq, mcols, p, st)
+                            : launch_bwd_main_t<D, BF16, false, false, true>(mq, mk, mv, mdo, mdq, mcols, p, st));
   if (varlen)
     return causal ? launch_bwd_main_t<D, BF16, true, true>(mq, mk, mv, mdo, mdq, mcols, p, st)
                   : launch_bwd_main_t<D, BF16, false, true>(mq, mk, mv, mdo, mdq, mcols, p, st);
@@ -650,6 +654,27 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                 (size_t)FA_BWD_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+fa_status fa_fwd_varlen_dropout(const void* q, const void* k, const void* v, void* o, float* lse,
+                                const int* cu_seqlens, int nseq, int max_seqlen, int total, int H, int D, float scale,
+                                int causal, fa_dtype dt, float dropout_p, uint64_t seed, uint64_t offset,
+                                void* stream) {
+  if (!dropout_p_ok(dropout_p)) return FA_ERR_INVALID_ARG;
+  if (dropout_p == 0.f)
+    return fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, nseq, max_seqlen, total, H, D, scale, causal, dt, stream);
+  if (nseq < 0 || max_seqlen < 0 || total < 0 || H < 0) return FA_ERR_INVALID_ARG;
+  if (dt != FA_BF16 && dt != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (nseq == 0 || H == 0 || total == 0 || max_seqlen == 0) return FA_OK;
+  if (max_seqlen > total) return FA_ERR_INVALID_ARG;
+  if (!ptrs_ok({q, k, v, o, lse}) || !cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if ((long long)nseq * H > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  const fa::Dropout d = make_dropout(dropout_p, seed, offset);
+  return run_fwd(q, k, v, o, lse, cu_seqlens, H, max_seqlen, total, nseq, D, scale, causal != 0, dt == FA_BF16, true,
+                 static_cast<cudaStream_t>(stream), &d);
+}
+
 size_t fa_bwd_varlen_workspace_size(int nseq, int max_seqlen, int total, int H, int D) {
   if (nseq <= 0 || max_seqlen <= 0 || total <= 0 || H <= 0 || (D != 64 && D != 128)) return 0;
   return ws_layout(H, nseq, max_seqlen, total, D).total;
@@ -672,6 +697,32 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   const fa::BwdParams p = bwd_params(H, nseq, max_seqlen, total, cu_seqlens, D, scale, deterministic != 0,
                                      static_cast<uint8_t*>(workspace), dk, dv);
   return run_bwd(q, k, v, o, dO, lse, dq, p, D, causal != 0, dt == FA_BF16, true, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_bwd_varlen_dropout(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens, int nseq,
+                                int max_seqlen, int total, int H, int D, float scale, int causal, fa_dtype dt,
+                                int deterministic, float dropout_p, uint64_t seed, uint64_t offset, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!dropout_p_ok(dropout_p)) return FA_ERR_INVALID_ARG;
+  if (dropout_p == 0.f)
+    return fa_bwd_varlen(q, k, v, o, dO, lse, dq, dk, dv, cu_seqlens, nseq, max_seqlen, total, H, D, scale, causal,
+                         dt, deterministic, workspace, workspace_bytes, stream);
+  if (nseq < 0 || max_seqlen < 0 || total < 0 || H < 0) return FA_ERR_INVALID_ARG;
+  if (dt != FA_BF16 && dt != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (nseq == 0 || H == 0 || total == 0 || max_seqlen == 0) return FA_OK;
+  if (max_seqlen > total) return FA_ERR_INVALID_ARG;
+  if (!ptrs_ok({q, k, v, o, dO, lse, dq, dk, dv}) || !cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < ws_layout(H, nseq, max_seqlen, total, D).total) return FA_ERR_INVALID_ARG;
+  fa::BwdParams p = bwd_params(H, nseq, max_seqlen, total, cu_seqlens, D, scale, deterministic != 0,
+                               static_cast<uint8_t*>(workspace), dk, dv);
+  p.drop = make_dropout(dropout_p, seed, offset);
+  return run_bwd(q, k, v, o, dO, lse, dq, p, D, causal != 0, dt == FA_BF16, true, static_cast<cudaStream_t>(stream),
+                 true);
 }
 
 int fa_decode_num_splits(int B, int Hkv, int L_max) {

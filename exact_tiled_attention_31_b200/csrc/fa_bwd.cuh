@@ -647,10 +647,12 @@ __global__ void __launch_bounds__(512, 1)
         if constexpr (DROPOUT) {
           const uint32_t c4 = lane & 3u, th = p.drop.thresh;
           const uint32_t keyquad = (uint32_t)kv >> 2, qp0 = (uint32_t)(128 * i + 64 * half) >> 1;
+          // head word of the counter: b * H + h, a packed batch's sequence as b
+          const uint32_t mask_head = (uint32_t)(x.seq * p.heads + x.head);
           keep_lo = keep_hi = 0u;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const uint4 w = philox4x32_10(make_uint4(keyquad, qp0 + 8 * c4 + q, (uint32_t)x.head, p.drop.offset),
+            const uint4 w = philox4x32_10(make_uint4(keyquad, qp0 + 8 * c4 + q, mask_head, p.drop.offset),
                                           p.drop.seed_lo, p.drop.seed_hi);
             // key 4m + t: word (t >> 1) for the even query, 2 + (t >> 1) for
             // the odd one; half t & 1 of each; packed (even, odd) as 2 x 16 bits

@@ -40,7 +40,7 @@
 //               at the end, O / l and LSE to global.
 // TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
 // Fully masked causal tiles are never loaded or multiplied.
-// DROPOUT instances (dense batches) zero the dropped P values before they
+// DROPOUT instances (dense or packed batches) zero the dropped P values before they
 // are published for the P V product, from a Philox4x32-10 mask regenerated
 // from (head, query, key) indices, and scale O by 1 / (keep probability) at
 // the end; the sums that normalise O and give LSE stay those of the
@@ -407,12 +407,15 @@ __global__ void __launch_bounds__(768, 1)
         const bool odd = (lane & 1u) != 0;
         const uint32_t th = p.drop.thresh;
         const uint32_t rowpair = (uint32_t)row >> 1, kq0 = (uint32_t)kv0 >> 2;
+        // head word of the counter: b * H + h, with a packed batch's sequence
+        // as its b (row and key indices count from the sequence's start)
+        const uint32_t mask_head = (uint32_t)(seq * p.heads + head);
         auto keep16 = [th](uint32_t u) -> uint32_t {  // 16-bit decisions of keys 2t, 2t + 1
           return ((u & 0xFFFFu) < th ? 0x0000FFFFu : 0u) | ((u >> 16) < th ? 0xFFFF0000u : 0u);
         };
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint4 w = philox4x32_10(make_uint4(kq0 + k + (odd ? 8u : 0u), rowpair, (uint32_t)head, p.drop.offset),
+          const uint4 w = philox4x32_10(make_uint4(kq0 + k + (odd ? 8u : 0u), rowpair, mask_head, p.drop.offset),
                                         p.drop.seed_lo, p.drop.seed_hi);
           // word 2 * (row & 1) + ((key >> 1) & 1)
           const uint32_t own0 = odd ? w.z : w.x, own1 = odd ? w.w : w.y;  // this row

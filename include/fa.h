@@ -207,7 +207,8 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          int deterministic, void* stream);
 
 /*
- * Dropout on the attention probabilities (dense [B, H, S, D] batches).
+ * Dropout on the attention probabilities (dense [B, H, S, D] batches; packed
+ * batches below).
  * "Flash Attention 的算法设计原理", section "练习口述回答", lists dropout as a
  * branch to test on its own. Because the mask must be regenerated in the
  * backward rather than stored, it comes from a counter-based generator.
@@ -241,6 +242,27 @@ fa_status fa_bwd_dropout(const void* q, const void* k, const void* v, const void
                          const float* lse, void* dq, void* dk, void* dv, int B, int H, int S, int D, float scale,
                          int causal, fa_dtype dt, int deterministic, float dropout_p, uint64_t seed,
                          uint64_t offset, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Dropout on a packed batch of variable-length sequences: fa_fwd_varlen /
+ * fa_bwd_varlen with the dropout of fa_fwd_dropout / fa_bwd_dropout.  The
+ * pages name both branches ("Flash Attention 的算法设计原理", "练习口述回答") but
+ * no mask layout for a pack; sequence s takes the mask that batch index s of
+ * a dense batch would get (the counter's head word is s * H + h, query and
+ * key indices count from the sequence's first token), so a pack of equal
+ * lengths drops exactly what the dense [nseq, H, L, D] batch drops.
+ * Arguments: those of fa_fwd_varlen / fa_bwd_varlen plus dropout_p, seed,
+ * offset as for fa_fwd_dropout; dropout_p = 0 is exactly the plain call.
+ */
+fa_status fa_fwd_varlen_dropout(const void* q, const void* k, const void* v, void* o, float* lse,
+                                const int* cu_seqlens, int nseq, int max_seqlen, int total, int H, int D,
+                                float scale, int causal, fa_dtype dt, float dropout_p, uint64_t seed,
+                                uint64_t offset, void* stream);
+fa_status fa_bwd_varlen_dropout(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens, int nseq,
+                                int max_seqlen, int total, int H, int D, float scale, int causal, fa_dtype dt,
+                                int deterministic, float dropout_p, uint64_t seed, uint64_t offset, void* workspace,
+                                size_t workspace_bytes, void* stream);
 
 /*
  * Decode: one new query token per (sequence, query head) against a KV cache

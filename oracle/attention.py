@@ -78,6 +78,8 @@ __all__ = [
     "dropout_keep",
     "attention_forward_dropout",
     "attention_backward_dropout",
+    "varlen_forward_dropout",
+    "varlen_backward_dropout",
     "flop_count",
 ]
 
@@ -450,6 +452,46 @@ def attention_backward_dropout(q, k, v, do, scale: float, causal: bool, p: float
             t[n] = x
     if heads is None:
         return tuple(t.reshape(B, H, S, -1) for t in out)
+    return tuple(out)
+
+
+def varlen_forward_dropout(q, k, v, cu_seqlens, scale: float, causal: bool, p: float, seed: int, offset: int,
+                           heads=None):
+    """Packed [H, T, D] forward with dropout on P.
+
+    Reading (the pages give no packed layout for the mask): sequence s of the
+    pack takes the mask a dense batch would give its batch index s, i.e.
+    head index s * H + h, query and key indices counted from the sequence's
+    own first token.  A pack of equal lengths therefore drops exactly what
+    the dense [nseq, H, L, D] batch drops.
+    """
+    q, k, v = to_f64(q), to_f64(k), to_f64(v)
+    H, T, D = q.shape
+    heads = list(range(H)) if heads is None else list(heads)
+    o = np.zeros((len(heads), T, v.shape[-1]))
+    lse = np.zeros((len(heads), T))
+    for n, h in enumerate(heads):
+        for si, (a, b) in enumerate(_seq_bounds(cu_seqlens)):
+            L = b - a
+            keep = dropout_keep(si * H + h, np.arange(L), np.arange(L), p, seed, offset)
+            o[n, a:b], lse[n, a:b] = _head_dropout(q[h, a:b], k[h, a:b], v[h, a:b], None, scale, causal, p, keep)
+    return o, lse
+
+
+def varlen_backward_dropout(q, k, v, do, cu_seqlens, scale: float, causal: bool, p: float, seed: int, offset: int,
+                            heads=None):
+    """dQ, dK, dV of a packed [H, T, D] batch with the mask of varlen_forward_dropout."""
+    q, k, v, do = to_f64(q), to_f64(k), to_f64(v), to_f64(do)
+    H, T, D = q.shape
+    heads = list(range(H)) if heads is None else list(heads)
+    out = [np.zeros((len(heads), T, D)) for _ in range(2)] + [np.zeros((len(heads), T, v.shape[-1]))]
+    for n, h in enumerate(heads):
+        for si, (a, b) in enumerate(_seq_bounds(cu_seqlens)):
+            L = b - a
+            keep = dropout_keep(si * H + h, np.arange(L), np.arange(L), p, seed, offset)
+            g = _head_dropout(q[h, a:b], k[h, a:b], v[h, a:b], do[h, a:b], scale, causal, p, keep)
+            for t, x in zip(out, g):
+                t[n, a:b] = x
     return tuple(out)
 
 

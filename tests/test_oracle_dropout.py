@@ -240,3 +240,50 @@ def test_planted_head_independent_mask_is_detected():
     q2, k2, v2 = (np.concatenate([x, x], axis=1) for x in (q, k, v))
     o, _ = oa.attention_forward_dropout(q2, k2, v2, 0.3, False, 0.5, seed=3, offset=0)
     assert np.abs(o[0, 0] - o[0, 1]).max() > 1e-3
+
+
+def test_packed_dropout_equals_dense_for_equal_lengths():
+    """A pack of equal-length sequences drops exactly what the dense batch
+    of the same shape drops (sequence s takes batch index s), so its O, LSE
+    and gradients equal the dense ones."""
+    g = np.random.default_rng(4)
+    nseq, H, L, D = 3, 2, 20, 8
+    q, k, v, do = (g.standard_normal((nseq, H, L, D)) for _ in range(4))
+    packed = [x.transpose(1, 0, 2, 3).reshape(H, nseq * L, D) for x in (q, k, v, do)]
+    cu = np.arange(nseq + 1) * L
+    for causal in (False, True):
+        o_d, l_d = oa.attention_forward_dropout(q, k, v, 0.3, causal, 0.4, seed=9, offset=2)
+        o_p, l_p = oa.varlen_forward_dropout(*packed[:3], cu, 0.3, causal, 0.4, seed=9, offset=2)
+        assert np.allclose(o_p, o_d.transpose(1, 0, 2, 3).reshape(H, nseq * L, D), atol=1e-13)
+        assert np.allclose(l_p, l_d.transpose(1, 0, 2).reshape(H, nseq * L), atol=1e-13)
+        g_d = oa.attention_backward_dropout(q, k, v, do, 0.3, causal, 0.4, seed=9, offset=2)
+        g_p = oa.varlen_backward_dropout(*packed, cu, 0.3, causal, 0.4, seed=9, offset=2)
+        for a, b in zip(g_p, g_d):
+            assert np.allclose(a, b.transpose(1, 0, 2, 3).reshape(H, nseq * L, D), atol=1e-12)
+
+
+def test_packed_dropout_p0_is_plain_and_sequences_get_their_own_masks():
+    """p = 0 is plain packed attention; two sequences of one pack with the
+    same inputs get different outputs (their masks differ), and a planted
+    mistake (every sequence reusing sequence 0's mask) makes them equal."""
+    g = np.random.default_rng(5)
+    H, L, D = 2, 24, 8
+    q1, k1, v1 = (g.standard_normal((H, L, D)) for _ in range(3))
+    q, k, v = (np.concatenate([x, x], axis=1) for x in (q1, k1, v1))
+    cu = np.array([0, L, 2 * L])
+    o0, l0 = oa.varlen_forward_dropout(q, k, v, cu, 0.3, True, 0.0, seed=1, offset=0)
+    o_ref, l_ref = oa.varlen_forward(q, k, v, cu, 0.3, True)
+    assert np.allclose(o0, o_ref, atol=1e-13) and np.allclose(l0, l_ref, atol=1e-13)
+    o, _ = oa.varlen_forward_dropout(q, k, v, cu, 0.3, True, 0.5, seed=1, offset=0)
+    assert not np.allclose(o[:, :L], o[:, L:])
+    real = oa.dropout_keep
+
+    def same_for_all_sequences(bh, rows, cols, p, seed, offset):
+        return real(bh % H, rows, cols, p, seed, offset)
+
+    oa.dropout_keep = same_for_all_sequences
+    try:
+        o_bad, _ = oa.varlen_forward_dropout(q, k, v, cu, 0.3, True, 0.5, seed=1, offset=0)
+    finally:
+        oa.dropout_keep = real
+    assert np.allclose(o_bad[:, :L], o_bad[:, L:])
