@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--sustained-s", type=float, default=2.0,
+                    help="seconds of back-to-back steps for the sustained leg (0 runs a single step)")
     return ap.parse_args()
 
 
@@ -470,7 +472,7 @@ def main():
 
     # ---- sustained: the same step back to back (no flush in between) for
     # about two seconds, clocks sampled over the whole run
-    sus_n = max(1, int(2.0 / max(1e-4, statistics.mean(e[0].elapsed_time(e[4]) for e in evs) * 1e-3)))
+    sus_n = max(1, int(args.sustained_s / max(1e-4, statistics.mean(e[0].elapsed_time(e[4]) for e in evs) * 1e-3)))
     sus_e0, sus_e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
