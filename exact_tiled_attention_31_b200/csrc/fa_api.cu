@@ -483,12 +483,12 @@ fa_status launch_decode_t(const fa::DecParams& p, cudaStream_t st) {
 // (the inverse of the exact keep probability t / 2^16); p in (0, 1).
 fa::Dropout make_dropout(float p, uint64_t seed, uint64_t offset) {
   fa::Dropout d;
-  const double t = std::max(1.0, std::floor((1.0 - (double)p) * 65536.0));
+  const double t = std::max(1.0, std::floor((1.0 - (double)p) * 256.0));
   d.thresh = (uint32_t)t;
   d.seed_lo = (uint32_t)seed;
   d.seed_hi = (uint32_t)(seed >> 32);
   d.offset = (uint32_t)offset;
-  d.scale = (float)(65536.0 / t);
+  d.scale = (float)(256.0 / t);
   return d;
 }
 

@@ -403,8 +403,12 @@ __global__ void __launch_bounds__(512, 1)
   auto region_x = [](uint32_t g) -> uint32_t { return (g & 1) ? C::TM_B : C::TM_A; };
 
   // register split over 512 threads launched with 128 each (65536):
-  // 128 x 56 (warps 0-3) + 256 x 136 (P/dS) + 128 x 176 (dQ) = 64512.
+  // 128 x 56 (warps 0-3) + 256 x RP (P/dS) + 128 x RQ (dQ), with (RP, RQ) =
+  // (136, 176) = 64512, and (144, 168) = 65536 for dropout, whose dS phase
+  // keeps the keep bits and D_i live as well.
   // Each warpgroup changes its budget inside its own branch.
+  constexpr int RP = DROPOUT ? 144 : 136, RQ = DROPOUT ? 168 : 176;
+  static_assert(128 * 56 + 256 * RP + 128 * RQ <= 65536, "register split");
   if (warp < 4) {
   regs_dec<56>();
   if (warp == 0) {
@@ -581,7 +585,7 @@ __global__ void __launch_bounds__(512, 1)
     __syncwarp();
   }
   } else if (warp < 12) {
-    regs_inc<136>();
+    regs_inc<RP>();
     // ------------------------------------------------------------ P / dS
     // One thread per key row and half of the 128 query columns: warps 4-7
     // take queries 0-63, warps 8-11 queries 64-127.  P and dS are
@@ -600,6 +604,52 @@ __global__ void __launch_bounds__(512, 1)
       bwd_decode<CAUSAL, VARLEN>(p, u, x);
       const int kv = 128 * x.j + r;  // key row inside the sequence
       const bool kv_valid = kv < x.seq_len;
+      // Dropout keep decisions of this key row against the half's 64 query
+      // columns of tile iq, pair-packed: queries 2e, 2e + 1 at bits
+      // pair_slot(e & 15), pair_slot(e & 15) + 8 of keep[e >> 4].  One Philox
+      // call covers query pair e x key octet (8m .. 8m + 7), one byte per
+      // element, and a key octet sits in eight consecutive lanes: lane 8m + c
+      // draws query pairs 4c .. 4c + 3, and each lane hands every other lane
+      // of its octet that lane's bytes of two calls at a time (XOR shuffles
+      // over the octet).  Drawn for the next step while this step's products
+      // run, so the generator stays off the critical path of P and dS.
+      uint32_t keep[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
+      auto make_keep = [&](int iq) {
+        const uint32_t c8 = lane & 7u;
+        const uint32_t t4 = p.drop.thresh * 0x01010101u, t4lo = t4 & 0x7f7f7f7fu;
+        const uint32_t keyoct = (uint32_t)kv >> 3, qp0 = (uint32_t)(128 * iq + 64 * half) >> 1;
+        // head word of the counter: b * H + h, a packed batch's sequence as b
+        const uint32_t mask_head = (uint32_t)(x.seq * p.heads + x.head);
+        uint32_t k0 = 0u, k1 = 0u;
+#pragma unroll
+        for (int q = 0; q < 4; q += 2) {
+          const uint4 w0 = philox4x32_10(make_uint4(keyoct, qp0 + 4 * c8 + q, mask_head, p.drop.offset),
+                                         p.drop.seed_lo, p.drop.seed_hi);
+          const uint4 w1 = philox4x32_10(make_uint4(keyoct, qp0 + 4 * c8 + q + 1, mask_head, p.drop.offset),
+                                         p.drop.seed_lo, p.drop.seed_hi);
+          // key 8m + t: byte t & 3 of word (t >> 2) for the even query and of
+          // word 2 + (t >> 2) for the odd one; the bytes of both calls packed
+          // as (even q, odd q, even q + 1, odd q + 1)
+          auto vals_for = [&w0, &w1](uint32_t t) -> uint32_t {
+            const uint32_t sh = 8u * (t & 3u);
+            const uint32_t e0 = (t & 4u) ? w0.y : w0.x, o0 = (t & 4u) ? w0.w : w0.z;
+            const uint32_t e1 = (t & 4u) ? w1.y : w1.x, o1 = (t & 4u) ? w1.w : w1.z;
+            return ((e0 >> sh) & 0xFFu) | (((o0 >> sh) & 0xFFu) << 8) | (((e1 >> sh) & 0xFFu) << 16) |
+                   (((o1 >> sh) & 0xFFu) << 24);
+          };
+#pragma unroll
+          for (uint32_t d = 0; d < 8; ++d) {
+            const uint32_t v = d == 0 ? vals_for(c8) : __shfl_xor_sync(0xffffffffu, vals_for(c8 ^ d), (int)d);
+            const uint32_t e = 4u * (c8 ^ d) + (uint32_t)q;  // query pairs e, e + 1 drawn by lane c8 ^ d
+            const uint32_t bits = pair_bits(bytes_below(v, t4, t4lo)) << ((e & 7u) + 16u * ((e >> 3) & 1u));
+            k0 |= (e & 16u) ? 0u : bits;
+            k1 |= (e & 16u) ? bits : 0u;
+          }
+        }
+        keep[0] = k0;
+        keep[1] = k1;
+      };
+      if constexpr (DROPOUT) make_keep(x.i_begin);
       for (int st = 0; st < x.n_steps; ++st, ++g) {
         const int i = x.i_begin + st;
         const int qs = g & 1;
@@ -637,46 +687,13 @@ __global__ void __launch_bounds__(512, 1)
           }
           pk[e] = pack2<BF16>(p0, p1);
         }
-        // dropout keep masks of the 64 query columns: bit e of keep_lo / keep_hi
-        // for queries 2e and 2e + 1 of this half.  One Philox call covers query
-        // pair e x key quad (4m .. 4m + 3), 16 bits per element, and a key quad
-        // sits in four consecutive lanes: lane 4m + c draws query pairs
-        // 8c .. 8c + 7, and each lane hands every other lane of its quad that
-        // lane's two 16-bit values (XOR shuffles over the quad).
-        uint32_t keep_lo = 0xFFFFFFFFu, keep_hi = 0xFFFFFFFFu;
-        if constexpr (DROPOUT) {
-          const uint32_t c4 = lane & 3u, th = p.drop.thresh;
-          const uint32_t keyquad = (uint32_t)kv >> 2, qp0 = (uint32_t)(128 * i + 64 * half) >> 1;
-          // head word of the counter: b * H + h, a packed batch's sequence as b
-          const uint32_t mask_head = (uint32_t)(x.seq * p.heads + x.head);
-          keep_lo = keep_hi = 0u;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint4 w = philox4x32_10(make_uint4(keyquad, qp0 + 8 * c4 + q, mask_head, p.drop.offset),
-                                          p.drop.seed_lo, p.drop.seed_hi);
-            // key 4m + t: word (t >> 1) for the even query, 2 + (t >> 1) for
-            // the odd one; half t & 1 of each; packed (even, odd) as 2 x 16 bits
-            auto vals_for = [&w](uint32_t t) -> uint32_t {
-              const uint32_t we = (t & 2u) ? w.y : w.x, wo = (t & 2u) ? w.w : w.z;
-              return (t & 1u) ? ((we >> 16) | (wo & 0xFFFF0000u)) : ((we & 0xFFFFu) | (wo << 16));
-            };
-#pragma unroll
-            for (uint32_t d = 0; d < 4; ++d) {
-              const uint32_t v = d == 0 ? vals_for(c4) : __shfl_xor_sync(0xffffffffu, vals_for(c4 ^ d), (int)d);
-              const uint32_t e = 8u * (c4 ^ d) + (uint32_t)q;  // query pair drawn by lane c4 ^ d
-              keep_lo |= ((v & 0xFFFFu) < th ? 1u : 0u) << e;
-              keep_hi |= ((v >> 16) < th ? 1u : 0u) << e;
-            }
-          }
-        }
         // P^T pairs go to columns [64*half, 64*half + 32) of X (inside this
         // half's own score columns, already read); with dropout the dV operand
         // is P * M (dV is scaled by s = 1 / keep probability at the end)
         if constexpr (DROPOUT) {
           uint32_t pd[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            pd[e] = pk[e] & (((keep_lo >> e) & 1u ? 0x0000FFFFu : 0u) | ((keep_hi >> e) & 1u ? 0xFFFF0000u : 0u));
+          for (int e = 0; e < 32; ++e) pd[e] = pk[e] & pair_keep_halves(keep[e >> 4], e & 15);
           tmem_st32(tX + 64 * half, pd);
         } else {
           tmem_st32(tX + 64 * half, pk);
@@ -699,28 +716,36 @@ __global__ void __launch_bounds__(512, 1)
         tmem_ld_wait(dv[1]);
         tc_fence_before();
         mbar_arrive(dp_taken);
+        BWD_TRACE(tw, 3700 + g);
         uint32_t dd[32];
         if constexpr (DROPOUT) {
-          // dP'^T = dPd^T - D (extra K step).  Kept: dS = P (dPd s - D)
-          // = P (dP' s + D (s - 1)); dropped: dS = -P D  (s = 1 / keep probability).
-          // D_i of the query rows comes from their per-query row (-D in three
-          // bf16 parts, columns 9-11) in shared memory.
+          // dP'^T = dPd^T - D (extra K step).  dS = P (M s dPd - D) with
+          // M s = m (s = 1 / keep probability for a kept element, 0 for a
+          // dropped one): dS = P (m (dP' + D) - D).  D_i of the half's 64
+          // query columns comes from their per-query rows (-D in three bf16
+          // parts, columns 9-11) in shared memory: lane l reads those of
+          // columns l and 32 + l, and hands them round.
           const uint8_t* ct = smem + C::CT_OFF + qs * 4096;
-          const float rp = p.drop.scale, rp1 = p.drop.scale - 1.f;
+          const float rp = p.drop.scale;
+          float d_l[2];
+#pragma unroll
+          for (int w2 = 0; w2 < 2; ++w2) {
+            const uint32_t qrow = (uint32_t)(64 * half + 32 * w2) + lane;
+            const uint2 c = *reinterpret_cast<const uint2*>(ct + swz32(qrow * 32u + 16u));
+            d_l[w2] = -(__uint_as_float(c.x & 0xFFFF0000u) + __uint_as_float(c.y << 16) +
+                        __uint_as_float(c.y & 0xFFFF0000u));
+          }
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const uint32_t* src = dv[e >> 4] + 2 * (e & 15);
-            float dq[2];
-#pragma unroll
-            for (int w2 = 0; w2 < 2; ++w2) {
-              const uint32_t qrow = (uint32_t)(64 * half + 2 * e + w2);
-              const uint2 c = *reinterpret_cast<const uint2*>(ct + swz32(qrow * 32u + 16u));
-              dq[w2] = -(__uint_as_float(c.x & 0xFFFF0000u) + __uint_as_float(c.y << 16) +
-                         __uint_as_float(c.y & 0xFFFF0000u));
-            }
+            // query columns 2e, 2e + 1 of the half
+            const float d0 = __shfl_sync(0xffffffffu, d_l[e >> 4], (2 * e) & 31);
+            const float d1 = __shfl_sync(0xffffffffu, d_l[e >> 4], (2 * e + 1) & 31);
+            const uint32_t kb = keep[e >> 4] >> pair_slot(e & 15);
+            const float m0 = (kb & 1u) ? rp : 0.f, m1 = (kb & 0x100u) ? rp : 0.f;
             const float2 pw = unpack2<BF16>(pk[e]);
-            const float a = pw.x * (((keep_lo >> e) & 1u) ? fmaf(__uint_as_float(src[0]), rp, dq[0] * rp1) : -dq[0]);
-            const float b = pw.y * (((keep_hi >> e) & 1u) ? fmaf(__uint_as_float(src[1]), rp, dq[1] * rp1) : -dq[1]);
+            const float a = pw.x * fmaf(m0, __uint_as_float(src[0]) + d0, -d0);
+            const float b = pw.y * fmaf(m1, __uint_as_float(src[1]) + d1, -d1);
             dd[e] = pack2<BF16>(a, b);
           }
         } else {
@@ -732,6 +757,7 @@ __global__ void __launch_bounds__(512, 1)
             dd[e] = pack2<BF16>(a, b);
           }
         }
+        BWD_TRACE(tw, 3500 + g);
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           // dS row r (key), 32 query columns: MN-major A operand of dQ = dS K,
@@ -751,6 +777,9 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_before();
         mbar_arrive(ds_full);
         BWD_TRACE(tw, 1600 + 4 * g + 3);
+        if constexpr (DROPOUT)
+          if (st + 1 < x.n_steps) make_keep(i + 1);
+        BWD_TRACE(tw, 3300 + g);
       }
       if (!ok) break;
       // ---- epilogue: dV and scale * dK rows of this key tile
@@ -784,7 +813,7 @@ __global__ void __launch_bounds__(512, 1)
       tc_fence_before();
     }
   } else {
-    regs_inc<176>();
+    regs_inc<RQ>();
     // ------------------------------------------------------------ dQ (one thread per query row)
     const int c = threadIdx.x - 384;                 // query row within the tile = TMEM lane
     const int wq = warp - 12;                        // this warp's 32 rows: 32*wq ..

@@ -325,6 +325,42 @@ __global__ void __launch_bounds__(768, 1)
     float* my_max = pmax_buf + (2 * t + h) * 128 + r;
     const float* other_max = pmax_buf + (2 * t + (h ^ 1)) * 128 + r;
     float m = -INFINITY, l = 0.f, lr = 0.f;
+    // Dropout keep decisions of this row's 64 keys of one step, pair-packed:
+    // keys 2i, 2i + 1 of the half's first 32 at bits pair_slot(i),
+    // pair_slot(i) + 8 of keep[0], the next 32 in keep[1].  One Philox call
+    // covers rows (2m, 2m + 1) x key octet o (one byte per element: byte
+    // key & 3 of word 2 (row & 1) + ((key >> 2) & 1)), and rows 2m, 2m + 1
+    // sit in the two lanes of a pair: the even lane draws the half's octets
+    // 0-3, the odd lane 4-7, and each hands the other row's two words
+    // across.  Drawn for step j + 1 while step j's products run, so the
+    // generator stays off the softmax's critical path.
+    uint32_t keep[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
+    auto make_keep = [&](int jj) {
+      const bool odd = (lane & 1u) != 0;
+      const uint32_t t4 = p.drop.thresh * 0x01010101u, t4lo = t4 & 0x7f7f7f7fu;
+      const uint32_t rowpair = (uint32_t)row >> 1, ko0 = (uint32_t)(128 * jj + 64 * h) >> 3;
+      // head word of the counter: b * H + h, with a packed batch's sequence
+      // as its b (row and key indices count from the sequence's start)
+      const uint32_t mask_head = (uint32_t)(seq * p.heads + head);
+      uint32_t k0 = 0u, k1 = 0u;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint4 w = philox4x32_10(make_uint4(ko0 + k + (odd ? 4u : 0u), rowpair, mask_head, p.drop.offset),
+                                      p.drop.seed_lo, p.drop.seed_hi);
+        const uint32_t own0 = odd ? w.z : w.x, own1 = odd ? w.w : w.y;  // this row
+        const uint32_t oth0 = odd ? w.x : w.z, oth1 = odd ? w.y : w.w;  // the partner row
+        const uint32_t got0 = __shfl_xor_sync(0xffffffffu, oth0, 1), got1 = __shfl_xor_sync(0xffffffffu, oth1, 1);
+        // keys 8k .. 8k + 3 are pairs 4k, 4k + 1; keys 8k + 4 .. are 4k + 2, 4k + 3
+        k0 |= (pair_bits(bytes_below(odd ? got0 : own0, t4, t4lo)) << pair_slot(4 * k)) |
+              (pair_bits(bytes_below(odd ? got1 : own1, t4, t4lo)) << pair_slot(4 * k + 2));  // octet k
+        k1 |= (pair_bits(bytes_below(odd ? own0 : got0, t4, t4lo)) << pair_slot(4 * k)) |
+              (pair_bits(bytes_below(odd ? own1 : got1, t4, t4lo)) << pair_slot(4 * k + 2));  // octet 4 + k
+      }
+      keep[0] = k0;
+      keep[1] = k1;
+    };
+    if constexpr (DROPOUT)
+      if (n_t > 0) make_keep(0);
     bool ok = true;
     for (int j = 0; j < n_t; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, FWD_SITE_S));
@@ -398,35 +434,12 @@ __global__ void __launch_bounds__(768, 1)
         pk[16 + i] = exp_pair(sv[1][2 * i], sv[1][2 * i + 1], fsum1, rsum1);
       }
       if constexpr (DROPOUT) {
-        // pk[2q], pk[2q + 1] hold keys kv0 + 4q .. +3.  One Philox call
-        // covers rows (2m, 2m + 1) x key quad q (16 bits per element), and
-        // rows 2m, 2m + 1 sit in lanes of one pair: the even lane draws quads
-        // 0-7, the odd lane 8-15, and each hands the other row's two words
-        // across.  The sums above are of the undropped P (the softmax
-        // normaliser and LSE).
-        const bool odd = (lane & 1u) != 0;
-        const uint32_t th = p.drop.thresh;
-        const uint32_t rowpair = (uint32_t)row >> 1, kq0 = (uint32_t)kv0 >> 2;
-        // head word of the counter: b * H + h, with a packed batch's sequence
-        // as its b (row and key indices count from the sequence's start)
-        const uint32_t mask_head = (uint32_t)(seq * p.heads + head);
-        auto keep16 = [th](uint32_t u) -> uint32_t {  // 16-bit decisions of keys 2t, 2t + 1
-          return ((u & 0xFFFFu) < th ? 0x0000FFFFu : 0u) | ((u >> 16) < th ? 0xFFFF0000u : 0u);
-        };
+        // drop: pk[i] holds keys 2i, 2i + 1 of the half (pair slot i & 15 of
+        // keep[i >> 4])
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint4 w = philox4x32_10(make_uint4(kq0 + k + (odd ? 8u : 0u), rowpair, mask_head, p.drop.offset),
-                                        p.drop.seed_lo, p.drop.seed_hi);
-          // word 2 * (row & 1) + ((key >> 1) & 1)
-          const uint32_t own0 = odd ? w.z : w.x, own1 = odd ? w.w : w.y;  // this row
-          const uint32_t oth0 = odd ? w.x : w.z, oth1 = odd ? w.y : w.w;  // the partner row
-          const uint32_t got0 = __shfl_xor_sync(0xffffffffu, oth0, 1), got1 = __shfl_xor_sync(0xffffffffu, oth1, 1);
-          const uint32_t a0 = odd ? got0 : own0, a1 = odd ? got1 : own1;  // this row, quad k
-          const uint32_t b0 = odd ? own0 : got0, b1 = odd ? own1 : got1;  // this row, quad 8 + k
-          pk[2 * k] &= keep16(a0);
-          pk[2 * k + 1] &= keep16(a1);
-          pk[16 + 2 * k] &= keep16(b0);
-          pk[16 + 2 * k + 1] &= keep16(b1);
+        for (int i = 0; i < 16; ++i) {
+          pk[i] &= pair_keep_halves(keep[0], i);
+          pk[16 + i] &= pair_keep_halves(keep[1], i);
         }
       }
       tmem_st32(tS + 32 * h, pk);
@@ -444,6 +457,9 @@ __global__ void __launch_bounds__(768, 1)
       l = l * alpha + ((f0 + f1) + (f2_ + f3));
       lr = lr * alpha + ((r0 + r1) + (r2 + r3));
       m = m_new;
+      // the next step's keep bits, while the tensor core works on this step
+      if constexpr (DROPOUT)
+        if (j + 1 < n_t) make_keep(j + 1);
     }
     if (ok && n_t > 0) {
       sum_buf[((2 * t + h) * 2 + 0) * 128 + r] = l;

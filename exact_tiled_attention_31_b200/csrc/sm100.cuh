@@ -393,8 +393,8 @@ __device__ __forceinline__ void accum2(uint32_t v, float& s0, float& s1) {
 template <bool BF16>
 __device__ __forceinline__ float2 unpack2(uint32_t v) {
   if constexpr (BF16) {
-    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&v);
-    return __bfloat1622float2(h);
+    // bf16 -> fp32 is exact: the 16 bits become the top of the fp32 word
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
   } else {
     __half2 h = *reinterpret_cast<__half2*>(&v);
     return __half22float2(h);
@@ -447,12 +447,44 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
   return c;
 }
 
+// Four byte-wise keep decisions at once: the top bit of byte n of the result
+// is set when byte n of u is below t (1 <= t <= 255); the other bits carry
+// nothing.  t4 = t * 0x01010101, t4lo = t4 & 0x7f7f7f7f.  Per byte,
+// (u | 0x80) - (t & 0x7f) cannot borrow from the next byte, and its top bit
+// is set exactly when the low seven bits of u are at least those of t; so
+// u < t when u's top bit is clear and t's set, or the top bits agree and that
+// difference's top bit is clear.
+__device__ __forceinline__ uint32_t bytes_below(uint32_t u, uint32_t t4, uint32_t t4lo) {
+  const uint32_t x = (u | 0x80808080u) - t4lo;
+  return (~u & t4) | (~(u ^ t4) & ~x);
+}
+// The byte decisions of bytes_below packed for pairs: byte 0's at bit 0,
+// byte 2's at bit 1, byte 1's at bit 8 and byte 3's at bit 9.
+__device__ __forceinline__ uint32_t pair_bits(uint32_t w) {
+  const uint32_t y = (w & 0x80808080u) >> 7;
+  return (y | (y >> 15)) & 0x0303u;
+}
+// Bit of pair slot i (0..15) of a pair-packed word: the first element of
+// pair i at bit pair_slot(i), the second at pair_slot(i) + 8.
+__device__ __forceinline__ constexpr int pair_slot(int i) { return (i & 7) + 16 * (i >> 3); }
+// Halfword keep masks of pair slot i of a pair-packed word x: the low
+// halfword is 0xFFFF when the first element is kept, the high one when the
+// second is (prmt with sign replication from bits 7 and 15).  i is a
+// compile-time constant at every call (unrolled loops), so the shift folds.
+__device__ __forceinline__ uint32_t pair_keep_halves(uint32_t x, int i) {
+  const int b = pair_slot(i);
+  const uint32_t y = b <= 7 ? x << (7 - b) : x >> (b - 7);
+  uint32_t m;
+  asm("prmt.b32 %0, %1, %1, 0x9988;" : "=r"(m) : "r"(y));
+  return m;
+}
+
 // Dropout parameters shared by the forward and backward kernels.  Element
-// (head bh, query i, key j) is kept when half (j & 1) (low for even j) of
-// word 2 (i & 1) + ((j >> 1) & 1) of Philox4x32-10 at counter (j >> 2,
-// i >> 1, bh, offset), key (seed_lo, seed_hi), is below `thresh` =
-// max(1, floor((1 - p) 2^16)); kept values are scaled by `scale` =
-// 2^16 / thresh, the inverse of the exact keep probability.
+// (head bh, query i, key j) is kept when byte (j & 3) of word
+// 2 (i & 1) + ((j >> 2) & 1) of Philox4x32-10 at counter (j >> 3, i >> 1,
+// bh, offset), key (seed_lo, seed_hi), is below `thresh` =
+// max(1, floor((1 - p) 2^8)); kept values are scaled by `scale` =
+// 2^8 / thresh, the inverse of the exact keep probability.
 struct Dropout {
   uint32_t thresh, seed_lo, seed_hi, offset;
   float scale;

@@ -218,11 +218,12 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
  *
  * The mask M[b,h,i,j] comes from Philox4x32-10 (Salmon et al., "Parallel
  * random numbers: as easy as 1, 2, 3", SC 2011):
- *   - counter (j >> 2, i >> 1, b*H + h, offset mod 2^32);
+ *   - counter (j >> 3, i >> 1, b*H + h, offset mod 2^32);
  *   - key (seed mod 2^32, seed >> 32);
- *   - word 2*(i & 1) + ((j >> 1) & 1), low half for even j, high half for odd j.
- * M = 1 when that 16-bit value is below t = max(1, floor((1 - p) * 2^16)).
- * An element is therefore kept with probability t / 2^16, and s = 2^16 / t
+ *   - word 2*(i & 1) + ((j >> 2) & 1), byte j & 3 of it (bits 8(j & 3) ..).
+ * M = 1 when that byte is below t = max(1, floor((1 - p) * 2^8)).
+ * An element is therefore kept with probability t / 2^8 (dropout_p is taken
+ * to the smallest multiple of 2^-8 that is not below it), and s = 2^8 / t
  * keeps E[O] exact.
  * fa_bwd_dropout, given the same (dropout_p, seed, offset), regenerates M.
  * It returns the gradients of sum(dO * O) for that O:

@@ -338,19 +338,20 @@ def merge_partials(o_parts, lse_parts):
 # pages fix neither the generator nor where the mask sits, so the reading is:
 #
 # * P is the exact softmax; the output uses  Pd = P * M * s  with M_ij in
-#   {0, 1} (kept with probability t / 2^16, t below) and s = 2^16 / t;
+#   {0, 1} (kept with probability t / 2^8, t below) and s = 2^8 / t;
 #   O = Pd V.  LSE is the statistic of the undropped softmax (dropout comes
 #   after normalisation).
-# * M_ij for head bh (= b * H + h), query i, key j is decided by 16 bits of
+# * M_ij for head bh (= b * H + h), query i, key j is decided by one byte of
 #   one Philox4x32-10 output (Salmon, Moraes, Dror and Shaw, "Parallel random
 #   numbers: as easy as 1, 2, 3", SC 2011) with
-#       counter = (j >> 2, i >> 1, bh, offset mod 2^32),
+#       counter = (j >> 3, i >> 1, bh, offset mod 2^32),
 #       key     = (seed mod 2^32, seed >> 32 mod 2^32):
-#   word number 2 * (i & 1) + ((j >> 1) & 1), its low half for even j and its
-#   high half for odd j.  The element is kept when that 16-bit value is below
-#   t = floor((1 - p) * 2^16) (t >= 1), so an element is kept with
-#   probability t / 2^16 exactly, and kept values are scaled by 2^16 / t,
-#   which keeps E[O] = O exactly.  One call covers a 2 x 4 (query, key) block.
+#   word number 2 * (i & 1) + ((j >> 2) & 1), byte j & 3 of it (the lowest
+#   for j & 3 = 0).  The element is kept when that byte is below
+#   t = floor((1 - p) * 2^8) (t >= 1), so an element is kept with
+#   probability t / 2^8 exactly (p is taken to the next multiple of 2^-8
+#   above it, or equal), and kept values are scaled by 2^8 / t, which keeps
+#   E[O] = O exactly.  One call covers a 2 x 8 (query, key) block.
 # * Backward of L = sum(dO * O) with the same M:
 #       dV = Pd^T dO,  dPd = dO V^T,  dP = dPd * M * s,
 #       D_i = sum_j P_ij dP_ij  (= dO_i . O_i),  dS = P * (dP - D),
@@ -385,26 +386,31 @@ def philox4x32_10(ctr, key):
 
 
 def dropout_keep_threshold(p: float) -> int:
-    """16-bit threshold t = max(1, floor((1 - p) 2^16)): a value below it keeps the element."""
+    """8-bit threshold t = max(1, floor((1 - p) 2^8)): a byte below it keeps the element."""
     if not 0.0 <= p < 1.0:
         raise ValueError("dropout probability must be in [0, 1)")
-    return max(1, int(np.floor((1.0 - p) * 65536.0)))
+    return max(1, int(np.floor((1.0 - p) * 256.0)))
 
 
 def dropout_scale(p: float) -> float:
-    """Scale of the kept values, 2^16 / t (1 / the exact keep probability); 1 for p = 0."""
-    return 65536.0 / dropout_keep_threshold(p)
+    """Scale of the kept values, 2^8 / t (1 / the exact keep probability); 1 for p = 0."""
+    return 256.0 / dropout_keep_threshold(p)
 
 
 def dropout_keep(bh: int, rows, cols, p: float, seed: int, offset: int) -> np.ndarray:
-    """Boolean keep mask [len(rows), len(cols)] of head bh (query rows, key columns)."""
+    """Boolean keep mask [len(rows), len(cols)] of head bh (query rows, key columns).
+
+    Element (i, j) reads byte (j & 3) of word 2 (i & 1) + ((j >> 2) & 1) of
+    Philox4x32-10 at counter (j >> 3, i >> 1, bh, offset), key (seed low,
+    seed high 32 bits): one call covers a 2 x 8 (query, key) block.
+    """
     i = np.asarray(rows, dtype=np.int64)[:, None]
     j = np.asarray(cols, dtype=np.int64)[None, :]
-    words = philox4x32_10((j >> 2, i >> 1, bh, offset & 0xFFFFFFFF), (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF))
-    sel = 2 * (i & 1) + ((j >> 1) & 1)
+    words = philox4x32_10((j >> 3, i >> 1, bh, offset & 0xFFFFFFFF), (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF))
+    sel = 2 * (i & 1) + ((j >> 2) & 1)
     w = np.choose(np.broadcast_to(sel, np.broadcast_shapes(i.shape, j.shape)), words).astype(np.int64)
-    half = np.where((j & 1) == 1, w >> 16, w & 0xFFFF)
-    return half < dropout_keep_threshold(p)
+    byte = (w >> (8 * (j & 3))) & 0xFF
+    return byte < dropout_keep_threshold(p)
 
 
 def _head_dropout(q, k, v, do, scale, causal, p, keep):
