@@ -631,11 +631,15 @@ __global__ void __launch_bounds__(512, 1)
           // word 2 + (t >> 2) for the odd one; the bytes of both calls packed
           // as (even q, odd q, even q + 1, odd q + 1)
           auto vals_for = [&w0, &w1](uint32_t t) -> uint32_t {
-            const uint32_t sh = 8u * (t & 3u);
             const uint32_t e0 = (t & 4u) ? w0.y : w0.x, o0 = (t & 4u) ? w0.w : w0.z;
             const uint32_t e1 = (t & 4u) ? w1.y : w1.x, o1 = (t & 4u) ? w1.w : w1.z;
-            return ((e0 >> sh) & 0xFFu) | (((o0 >> sh) & 0xFFu) << 8) | (((e1 >> sh) & 0xFFu) << 16) |
-                   (((o1 >> sh) & 0xFFu) << 24);
+            // byte t & 3 of e and of o, side by side, for each call; then both
+            const uint32_t sel = (t & 3u) | ((4u | (t & 3u)) << 4);
+            uint32_t a, b, r;
+            asm("prmt.b32 %0, %1, %2, %3;" : "=r"(a) : "r"(e0), "r"(o0), "r"(sel));
+            asm("prmt.b32 %0, %1, %2, %3;" : "=r"(b) : "r"(e1), "r"(o1), "r"(sel));
+            asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(a), "r"(b));
+            return r;
           };
 #pragma unroll
           for (uint32_t d = 0; d < 8; ++d) {
