@@ -36,6 +36,7 @@ DENSE = [  # (B, H, S, D, dtype, causal)
     (1, 32, 4096, 128, "fp16", True),
     (1, 32, 4096, 128, "bf16", False),
     (4, 16, 8192, 128, "bf16", True),
+    (1, 32, 32768, 128, "bf16", True),
 ]
 DECODE = [  # (B, Hq, Hkv, L, D)
     (8, 32, 8, 8192, 128),
