@@ -6,7 +6,8 @@ packed variable-length batches and decode.  One JSON line per row.
     python bench_table.py [--only dense,dropout,varlen,decode] [--iters N]
 
 Device time with CUDA events on the launching stream, at least 3 warm-up
-calls, the mean of ``--iters`` calls.  The forward/backward rows write a
+calls, the mean of ``--iters`` calls, queued behind a ~10 ms spin so that the
+host's launch overhead never shows in a short call's events.  The forward/backward rows write a
 256 MiB buffer (above the 126 MB L2) between calls, outside the event pairs;
 the decode rows alternate two input sets instead (each set's caches exceed
 L2).  FLOPs follow bench.py's convention (forward 4*S^2*D per head, halved
@@ -76,6 +77,9 @@ def main():
             fn(0)
         torch.cuda.synchronize()
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+        # keep the GPU busy while the host queues the timed calls, so a short
+        # call's events measure the device, not the host's launch overhead
+        torch.cuda._sleep(20_000_000)
         for i, (e0, e1) in enumerate(evs):
             if do_flush:
                 flush.zero_()

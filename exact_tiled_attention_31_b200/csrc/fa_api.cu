@@ -219,10 +219,18 @@ fa_status launch_bwd_pre(const void* o, const void* dO, const float* lse, const 
                          cudaStream_t st) {
   const uint16_t* o16 = static_cast<const uint16_t*>(o);
   const uint16_t* do16 = static_cast<const uint16_t*>(dO);
+  // y: (head, sequence) slices (looped past 65535); x: about eight blocks per
+  // SM in all, at least one, at most enough for one pass over a slice's rows
+  const long long slices = (long long)p.heads * p.nseq;
+  if ((long long)p.S_pad * (D / 8) + 31 > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;  // 32-bit row indices
+  const int gy = (int)std::min<long long>(slices, 65535);
+  const long long per_slice = ((long long)p.S_pad * (D / 8) + 255) / 256;
+  const int gx = (int)std::max<long long>(1, std::min<long long>(per_slice, (sm_count() * 8LL + gy - 1) / gy));
+  const dim3 grid(gx, gy);
   if (varlen)
-    fa::bwd_pre_kernel<D, BF16, true><<<sm_count() * 8, 256, 0, st>>>(o16, do16, lse, p);
+    fa::bwd_pre_kernel<D, BF16, true><<<grid, 256, 0, st>>>(o16, do16, lse, p);
   else
-    fa::bwd_pre_kernel<D, BF16, false><<<sm_count() * 8, 256, 0, st>>>(o16, do16, lse, p);
+    fa::bwd_pre_kernel<D, BF16, false><<<grid, 256, 0, st>>>(o16, do16, lse, p);
   g_launches.fetch_add(1);
   return from_cuda(cudaGetLastError());
 }

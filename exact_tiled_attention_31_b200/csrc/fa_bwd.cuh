@@ -179,73 +179,75 @@ __device__ __forceinline__ bool bwd_decode(const BwdParams& p, int u, BwdUnit& x
 
 // ---------------------------------------------------------------------------
 // bwd_pre: one group of D/8 lanes per row, 16-byte loads, shuffle reduction.
+// blockIdx.y walks the (head, sequence) slices and blockIdx.x the rows of a
+// slice, so a row's indices need no division by a runtime size.
 // ---------------------------------------------------------------------------
 template <int D, bool BF16, bool VARLEN>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dO,
                                                       const float* __restrict__ lse, BwdParams p) {
-  constexpr int G = D / 8;  // lanes per row
-  const long long work = (long long)p.heads * p.nseq * p.S_pad * G;
-  const long long bound = (work + 31) / 32 * 32;  // whole warps take the same trips
-  const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long nthreads = (long long)gridDim.x * blockDim.x;
-  for (long long idx = gtid; idx < bound; idx += nthreads) {
-    const bool in = idx < work;
-    const long long row = idx / G;  // padded row: (head * nseq + seq) * S_pad + s
-    const int part = (int)(idx % G);
-    const long long hs = in ? row / p.S_pad : 0;
-    const int h = (int)(hs / p.nseq);
-    const int seq = (int)(hs - (long long)h * p.nseq);
+  constexpr int G = D / 8;  // lanes per row (divides 32)
+  const int slices = p.heads * p.nseq;
+  const int work = p.S_pad * G;
+  const int bound = (work + 31) / 32 * 32;  // whole warps take the same trips
+  for (int slice = blockIdx.y; slice < slices; slice += gridDim.y) {
+    const int h = slice / p.nseq, seq = slice - h * p.nseq;
     int base = 0, len = p.S;
     if constexpr (VARLEN) {
       base = p.cu_seqlens[seq];
       len = p.cu_seqlens[seq + 1] - base;
     }
-    const int s = in ? (int)(row - hs * p.S_pad) : len;
-    const bool valid = s < len;
-    const size_t tok = (size_t)h * p.rows + base + s;  // token row in memory (valid rows only)
-    float acc = 0.f;
-    if (valid) {
-      const size_t off = tok * D + part * 8;
-      const uint4 a = *reinterpret_cast<const uint4*>(o + off);
-      const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
-      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < bound; idx += gridDim.x * blockDim.x) {
+      const bool in = idx < work;
+      const int s = in ? idx / G : len;  // padded row of the slice
+      const int part = idx % G;
+      const bool valid = s < len;
+      const size_t tok = (size_t)h * p.rows + base + s;  // token row in memory (valid rows only)
+      float acc = 0.f;
+      if (valid) {
+        const size_t off = tok * D + part * 8;
+        const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+        const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 x = unpack2<BF16>(av[i]), y = unpack2<BF16>(bv[i]);
-        acc = fmaf(x.x, y.x, acc);
-        acc = fmaf(x.y, y.y, acc);
+        for (int i = 0; i < 4; ++i) {
+          const float2 x = unpack2<BF16>(av[i]), y = unpack2<BF16>(bv[i]);
+          acc = fmaf(x.x, y.x, acc);
+          acc = fmaf(x.y, y.y, acc);
+        }
       }
-    }
-    // the G lanes of one row are consecutive lanes of one warp (G divides 32)
+      // the G lanes of one row are consecutive lanes of one warp
 #pragma unroll
-    for (int w = G / 2; w > 0; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
-    if (in && part == 0) {
-      // per-query row of the extra K step: the tensor core adds
-      // (1/(scale log2 e)) * (-LSE log2 e) to S^T and -D to dP^T
-      const float nl = valid ? lse[tok] * -1.4426950408889634f : -1e30f;
-      const float nd = valid ? -acc : 0.f;
-      float a[3], b[3];
-      a[0] = bf16_round(nl);
-      a[1] = valid ? bf16_round(nl - a[0]) : 0.f;
-      a[2] = valid ? bf16_round(nl - a[0] - a[1]) : 0.f;
-      b[0] = bf16_round(nd);
-      b[1] = bf16_round(nd - b[0]);
-      b[2] = bf16_round(nd - b[0] - b[1]);
-      float v[16];
+      for (int w = G / 2; w > 0; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
+      if (in && part == 0) {
+        // per-query row of the extra K step: the tensor core adds
+        // (1/(scale log2 e)) * (-LSE log2 e) to S^T and -D to dP^T
+        const float nl = valid ? lse[tok] * -1.4426950408889634f : -1e30f;
+        const float nd = valid ? -acc : 0.f;
+        float a[3], b[3];
+        a[0] = bf16_round(nl);
+        a[1] = valid ? bf16_round(nl - a[0]) : 0.f;
+        a[2] = valid ? bf16_round(nl - a[0] - a[1]) : 0.f;
+        b[0] = bf16_round(nd);
+        b[1] = bf16_round(nd - b[0]);
+        b[2] = bf16_round(nd - b[0] - b[1]);
+        float v[16];
 #pragma unroll
-      for (int k = 0; k < 9; ++k) v[k] = a[k % 3];
+        for (int k = 0; k < 9; ++k) v[k] = a[k % 3];
 #pragma unroll
-      for (int k = 0; k < 3; ++k) v[9 + k] = b[k];
+        for (int k = 0; k < 3; ++k) v[9 + k] = b[k];
 #pragma unroll
-      for (int k = 12; k < 16; ++k) v[k] = 0.f;
-      uint4* dst = reinterpret_cast<uint4*>(p.cols + (size_t)row * 16);
-      dst[0] = make_uint4(pack2<true>(v[0], v[1]), pack2<true>(v[2], v[3]), pack2<true>(v[4], v[5]),
-                          pack2<true>(v[6], v[7]));
-      dst[1] = make_uint4(pack2<true>(v[8], v[9]), pack2<true>(v[10], v[11]), pack2<true>(v[12], v[13]),
-                          pack2<true>(v[14], v[15]));
+        for (int k = 12; k < 16; ++k) v[k] = 0.f;
+        uint4* dst = reinterpret_cast<uint4*>(p.cols + ((size_t)slice * p.S_pad + s) * 16);
+        dst[0] = make_uint4(pack2<true>(v[0], v[1]), pack2<true>(v[2], v[3]), pack2<true>(v[4], v[5]),
+                            pack2<true>(v[6], v[7]));
+        dst[1] = make_uint4(pack2<true>(v[8], v[9]), pack2<true>(v[10], v[11]), pack2<true>(v[12], v[13]),
+                            pack2<true>(v[14], v[15]));
+      }
     }
   }
   // zero the dQ accumulator (16-byte stores) and the ordering counters
+  const long long nthreads = (long long)gridDim.x * gridDim.y * blockDim.x;
+  const long long gtid = ((long long)blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x;
   const long long n4 = (long long)p.heads * p.rows * D / 4;
   float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
   for (long long i = gtid; i < n4; i += nthreads) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
