@@ -63,12 +63,12 @@ def flops(w):
 # profiles/, with a digest of the kernel sources (code only) they were taken on.
 # Reported only while that code is unchanged (otherwise null: the counters are stale).
 NCU_TRAFFIC = {
-    "bwd_main": (289_733_083, "b447af11e5a0230dc9bf419b51b1e9859f9414e754d3bdd9bdf9bdc0af0f509c",
+    "bwd_main": (289_147_757, "4a155118eeec8dfe419a43060f2e8eb62f3a49f09fd57597c714c3c3fabfdc8d",
                  ("fa_bwd.cuh", "sm100.cuh")),
-    "fwd": (150_062_628, "07872b191dda19f5155567aaa8196f01d9cb90b24cf03519148bfdaef2daa18b",
+    "fwd": (150_075_867, "07872b191dda19f5155567aaa8196f01d9cb90b24cf03519148bfdaef2daa18b",
             ("fa_fwd.cuh", "sm100.cuh")),
     # decode split kernel, B8 Hq32 Hkv8 L8192 D128 bf16, 2 splits merged in-kernel (mean of 13 launches)
-    "decode": (268_679_876, "846d5a4899f92d94b763a91c821b7cccb1aff87d155460858407e160614621ed",
+    "decode": (268_688_265, "846d5a4899f92d94b763a91c821b7cccb1aff87d155460858407e160614621ed",
                ("fa_decode.cuh", "sm100.cuh")),
 }
 
