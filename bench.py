@@ -488,6 +488,19 @@ def main():
     fa.check_device_error()
     sus_ms = max_over_ranks({"s": sus_e0.elapsed_time(sus_e1) / sus_n}, device=dev)["s"]
 
+    # ---- warm L2: 20 steps back to back, each between its own events; the
+    # median (the L2 holds whatever the previous step left)
+    warm_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
+    barrier()
+    torch.cuda.synchronize()
+    for e0, e1 in warm_ev:
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    fa.check_device_error()
+    warm_ms = max_over_ranks({"w": statistics.median(a.elapsed_time(b) for a, b in warm_ev)}, device=dev)["w"]
+
     t_fwd = [e[0].elapsed_time(e[1]) for e in evs]
     t_pre = [e[1].elapsed_time(e[2]) for e in evs]
     t_main = [e[2].elapsed_time(e[3]) for e in evs]
@@ -600,6 +613,8 @@ def main():
 
     clocks = sampler.summary(clock_rows)
     sus_clocks = sampler.summary(clock_rows, sus_t0, sus_t1)
+    warm = {"steps": len(warm_ev), "median_ms_per_step": warm_ms, "value": job_tflops(world, f_fwd + f_bwd, warm_ms),
+            "unit": "TFLOP/s", "l2": "warm: steps back to back, no flush; median of 20"}
     sustained = {"steps": sus_n, "ms_per_step": sus_ms, "value": job_tflops(world, f_fwd + f_bwd, sus_ms),
                  "unit": "TFLOP/s", "l2": "not flushed (steps back to back)", "clocks": sus_clocks,
                  "ms_x_sm_mhz": sus_ms * (sus_clocks["sm_mhz"] or 0.0)}
@@ -617,7 +632,7 @@ def main():
             "fwd_bwd_pct_of_2250": 100 * fb_tf / DATASHEET_TFLOPS,
             "fwd_frac_of_measured": fwd_tf / pk["bf16_tflops"], "bwd_frac_of_measured": bwd_tf / pk["bf16_tflops"],
             "kernel_ms": ms, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches, "clocks": clocks, "sustained": sustained, "decode": decode,
+            "gpu_launches": launches, "clocks": clocks, "warm_l2": warm, "sustained": sustained, "decode": decode,
         }
         print(json.dumps(out), flush=True)
     if world > 1:
