@@ -471,6 +471,20 @@ def main():
     launches = fa.fa_launch_count() - launches0
     fa.check_device_error()
 
+    # ---- warm L2: 20 steps back to back, each between its own events; the
+    # median (the L2 holds whatever the previous step left).  Run before the
+    # sustained leg, which leaves the GPU at its power-capped clock.
+    warm_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
+    barrier()
+    torch.cuda.synchronize()
+    for e0, e1 in warm_ev:
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    fa.check_device_error()
+    warm_ms = max_over_ranks({"w": statistics.median(a.elapsed_time(b) for a, b in warm_ev)}, device=dev)["w"]
+
     # ---- sustained: the same step back to back (no flush in between) for
     # about two seconds, clocks sampled over the whole run
     sus_n = max(1, int(args.sustained_s / max(1e-4, statistics.mean(e[0].elapsed_time(e[4]) for e in evs) * 1e-3)))
@@ -488,18 +502,6 @@ def main():
     fa.check_device_error()
     sus_ms = max_over_ranks({"s": sus_e0.elapsed_time(sus_e1) / sus_n}, device=dev)["s"]
 
-    # ---- warm L2: 20 steps back to back, each between its own events; the
-    # median (the L2 holds whatever the previous step left)
-    warm_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
-    barrier()
-    torch.cuda.synchronize()
-    for e0, e1 in warm_ev:
-        e0.record(stream)
-        step()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    fa.check_device_error()
-    warm_ms = max_over_ranks({"w": statistics.median(a.elapsed_time(b) for a, b in warm_ev)}, device=dev)["w"]
 
     t_fwd = [e[0].elapsed_time(e[1]) for e in evs]
     t_pre = [e[1].elapsed_time(e[2]) for e in evs]
