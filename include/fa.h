@@ -283,11 +283,18 @@ fa_status fa_bwd_varlen_dropout(const void* q, const void* k, const void* v, con
  *            len_b are never read
  *   seq_lens [B] int32 in device memory (4-byte aligned)
  *   o        [B, Hq, D] 16-bit (dt);  lse [B, Hq] fp32, natural log
- *   n_splits number of key ranges each cache is cut into (1..1024).  Each
- *            range is reduced by its own CTA to a normalised partial O and
- *            its LSE in the workspace, and a second launch merges them:
+ *   n_splits number of key ranges each cache is cut into (1..1024), or 0.
+ *            Each range is reduced by its own CTA to a normalised partial O
+ *            and its LSE, and the parts are merged:
  *            LSE = log sum_s exp(LSE_s), O = sum_s exp(LSE_s - LSE) O_s.
- *            fa_decode_num_splits() returns the library's choice.
+ *            One range writes O and LSE directly; 2 to 4 ranges whose CTAs
+ *            fit in one wave merge inside the kernel (a thread-block cluster,
+ *            through distributed shared memory); otherwise the parts go to
+ *            the workspace and a second, dependent launch merges them.
+ *            0 ("balanced"): one CTA per SM, each running an equal share of
+ *            all caches' 32-key tiles (a share may end one cache and start
+ *            the next), one part per cache it meets, merged by the second
+ *            launch.  fa_decode_num_splits() returns the library's choice.
  *   workspace  device memory of at least fa_decode_workspace_size(B, Hq,
  *            n_splits, D) bytes, 256-byte aligned, owned by the caller; it
  *            may be reused once the call's work on `stream` has finished.
@@ -295,12 +302,17 @@ fa_status fa_bwd_varlen_dropout(const void* q, const void* k, const void* v, con
  * Requirements: D = 64 or 128; Hkv >= 1 with Hq a multiple of Hkv
  * (FA_ERR_INVALID_ARG otherwise) and G = Hq / Hkv <= 16 (FA_ERR_UNSUPPORTED
  * otherwise); B, Hkv <= 65535; q, k_cache, v_cache, o, lse 16-byte aligned.
- * B = 0 or Hq = 0 is a no-op.  Two kernel launches on `stream`.
+ * B = 0 or Hq = 0 is a no-op.  One or two kernel launches on `stream`.
  */
 /* The library's split count for fa_decode at these sizes (the key ranges of
  * "训练与推理价值"'s decode over a long cache; the pages give no rule, this one
  * is measured on B200). */
 int fa_decode_num_splits(int B, int Hkv, int L_max);
+/* Workspace bytes for fa_decode with these sizes: fp32 partial O and LSE per
+ * (sequence, query head, part); n_splits = 0 sizes balanced mode (B * Hq +
+ * 16384 part slots, independent of the cache length).  0 for unsupported
+ * arguments.  The two-phase size query of "ops-transformer里的FlashAttention",
+ * "ops-transformer里的完整算子". */
 size_t fa_decode_workspace_size(int B, int Hq, int n_splits, int D);
 fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, const int* seq_lens, void* o,
                     float* lse, int B, int Hq, int Hkv, int L_max, int D, float scale, fa_dtype dt,
