@@ -36,6 +36,10 @@
  *    waits too long on one of its internal barriers gives up, records
  *    FA_ERR_TIMEOUT in a per-device error word and exits; read it with
  *    fa_check_device_error().
+ *  - The compute calls may be recorded into a CUDA graph (stream capture)
+ *    once one call of the same kind has run outside the capture on the device
+ *    (it sets up per-device state); a replay reads the buffers as they are
+ *    then.  fa_check_device_error() synchronises and must stay outside.
  *  - No entry point falls back to another implementation: unsupported
  *    arguments return FA_ERR_UNSUPPORTED.
  */
