@@ -63,12 +63,12 @@ def flops(w):
 # profiles/, with a digest of the kernel sources (code only) they were taken on.
 # Reported only while that code is unchanged (otherwise null: the counters are stale).
 NCU_TRAFFIC = {
-    "bwd_main": (289_147_757, "4a155118eeec8dfe419a43060f2e8eb62f3a49f09fd57597c714c3c3fabfdc8d",
+    "bwd_main": (290_289_289, "38e7e701e3699f87901d35c1bedd4d82be544e1b4d3fe93cc960ed01b7519252",
                  ("fa_bwd.cuh", "sm100.cuh")),
-    "fwd": (150_075_867, "07872b191dda19f5155567aaa8196f01d9cb90b24cf03519148bfdaef2daa18b",
+    "fwd": (151_981_073, "60d40782546f254928a296b48e46227a32b0386512a60093b94047a7f3b88867",
             ("fa_fwd.cuh", "sm100.cuh")),
     # decode split kernel, B8 Hq32 Hkv8 L8192 D128 bf16, 2 splits merged in-kernel (mean of 13 launches)
-    "decode": (268_688_265, "846d5a4899f92d94b763a91c821b7cccb1aff87d155460858407e160614621ed",
+    "decode": (269_364_303, "94a39f624c60de04b4b8e9db037b53a1ad44dedd3f04b6f1889f98ec0dc51c8a",
                ("fa_decode.cuh", "sm100.cuh")),
 }
 
@@ -440,7 +440,7 @@ def main():
                            B, H, S, D, scale, causal, dt, 0, ws.data_ptr(), ws_bytes, sh), "fa_bwd_main")
         if ev:
             ev[3].record(stream)
-        chk(fa.fa_bwd_finish(dq.data_ptr(), B, H, S, D, scale, dt, ws.data_ptr(), ws_bytes, sh), "fa_bwd_finish")
+        chk(fa.fa_bwd_finish(dq.data_ptr(), B, H, S, D, scale, dt, 0, ws.data_ptr(), ws_bytes, sh), "fa_bwd_finish")
         if ev:
             ev[4].record(stream)
 

@@ -69,7 +69,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fa_bwd_preprocess.restype = i
     lib.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp, sz, vp]
     lib.fa_bwd_main.restype = i
-    lib.fa_bwd_finish.argtypes = [vp, i, i, i, i, f, i, vp, sz, vp]
+    lib.fa_bwd_finish.argtypes = [vp, i, i, i, i, f, i, i, vp, sz, vp]
     lib.fa_bwd_finish.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
     lib.fa_bwd_noalloc.restype = i
@@ -136,8 +136,9 @@ def fa_bwd_main(q, k, v, dO, dk, dv, B, H, S, D, scale, causal, dt, deterministi
                                       workspace, workspace_bytes, stream)
 
 
-def fa_bwd_finish(dq, B, H, S, D, scale, dt, workspace, workspace_bytes, stream) -> int:
-    return load_library().fa_bwd_finish(dq, B, H, S, D, scale, dt, workspace, workspace_bytes, stream)
+def fa_bwd_finish(dq, B, H, S, D, scale, dt, deterministic, workspace, workspace_bytes, stream) -> int:
+    return load_library().fa_bwd_finish(dq, B, H, S, D, scale, dt, int(deterministic), workspace, workspace_bytes,
+                                        stream)
 
 
 def fa_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, S, D, scale, causal, dt, deterministic,
@@ -405,7 +406,8 @@ def decode(q, k_cache, v_cache, seq_lens, scale: float | None = None, n_splits: 
 
 
 def check_device_error(stream=None):
-    """Synchronise and raise FAError if a kernel recorded a timeout."""
+    """Synchronise and raise FAError if a kernel recorded an error (a wait
+    that timed out, or split backward calls that disagreed on the mode)."""
     st = fa_check_device_error(_stream(stream))
     if st != FA_OK:
         raise FAError(st, "device")

@@ -179,10 +179,10 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 WsLayout ws_layout(long long heads, long long nseq, long long S, long long rows, int D) {
   const long long n_q = (S + 127) / 128, S_pad = n_q * 128;
   WsLayout w;
-  w.dq_acc = 0;
-  w.cols = up256((size_t)heads * rows * D * 4);
+  w.dq_acc = 0;  // two fp32 accumulators back to back (the second for deterministic mode)
+  w.cols = up256((size_t)2 * heads * rows * D * 4);
   w.sem = w.cols + up256((size_t)heads * nseq * S_pad * 32);
-  w.ticket = w.sem + up256((size_t)heads * nseq * n_q * 4);
+  w.ticket = w.sem + up256((size_t)heads * nseq * n_q * 2 * 4);
   w.total = w.ticket + 256;
   return w;
 }
@@ -235,19 +235,31 @@ fa_status launch_bwd_pre(const void* o, const void* dO, const float* lse, const 
   return from_cuda(cudaGetLastError());
 }
 
+template <int D, bool BF16, bool CAUSAL, bool VARLEN, bool DROPOUT, bool DET>
+fa_status launch_bwd_main_det(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                              const CUtensorMap& mdo, const CUtensorMap& mdq, const CUtensorMap& mcols,
+                              const fa::BwdParams& p, cudaStream_t st) {
+  using C = fa::BwdCfg<D>;
+  const int grid = std::min(p.units, sm_count());
+  if (set_smem<fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN, DROPOUT, DET>>(C::SMEM) != cudaSuccess)
+    return FA_ERR_CUDA;
+  fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN, DROPOUT, DET><<<(unsigned)grid, 512, C::SMEM, st>>>(
+      mq, mk, mv, mdo, mdq, mcols, p);
+  return FA_OK;
+}
+
 template <int D, bool BF16, bool CAUSAL, bool VARLEN, bool DROPOUT = false>
 fa_status launch_bwd_main_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const CUtensorMap& mdo, const CUtensorMap& mdq, const CUtensorMap& mcols,
                             const fa::BwdParams& p, cudaStream_t st) {
-  using C = fa::BwdCfg<D>;
   // persistent grid: at most one CTA per SM, each claiming units from the
   // workspace counter that bwd_pre zeroed
   if (p.units < 0) return FA_ERR_UNSUPPORTED;
   if (p.units == 0) return FA_OK;
-  const int grid = std::min(p.units, sm_count());
-  if (set_smem<fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN, DROPOUT>>(C::SMEM) != cudaSuccess) return FA_ERR_CUDA;
-  fa::bwd_main_kernel<D, BF16, CAUSAL, VARLEN, DROPOUT><<<(unsigned)grid, 512, C::SMEM, st>>>(mq, mk, mv, mdo, mdq,
-                                                                                           mcols, p);
+  const fa_status s = p.deterministic
+                          ? launch_bwd_main_det<D, BF16, CAUSAL, VARLEN, DROPOUT, true>(mq, mk, mv, mdo, mdq, mcols, p, st)
+                          : launch_bwd_main_det<D, BF16, CAUSAL, VARLEN, DROPOUT, false>(mq, mk, mv, mdo, mdq, mcols, p, st);
+  if (s != FA_OK) return s;
   g_launches.fetch_add(1);
   return from_cuda(cudaGetLastError());
 }
@@ -255,10 +267,18 @@ fa_status launch_bwd_main_t(const CUtensorMap& mq, const CUtensorMap& mk, const 
 template <int D, bool BF16>
 fa_status launch_bwd_main(const void* q, const void* k, const void* v, const void* dO, const fa::BwdParams& p,
                           bool causal, bool varlen, bool dropout, cudaStream_t st) {
+  if (p.deterministic) {
+    // the second accumulator (odd key tiles) starts at zero, and the flag
+    // tells bwd_post to add it
+    const size_t n = (size_t)p.heads * p.rows * D;
+    if (cudaMemsetAsync(p.dq_acc + n, 0, n * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(p.ticket + 1, 1, 1, st) != cudaSuccess)
+      return FA_ERR_CUDA;
+  }
   CUtensorMap mq, mk, mv, mdo, mdq, mcols;
   if (!make_map(&mq, q, D, p.rows, p.heads, BF16) || !make_map(&mk, k, D, p.rows, p.heads, BF16) ||
       !make_map(&mv, v, D, p.rows, p.heads, BF16) || !make_map(&mdo, dO, D, p.rows, p.heads, BF16) ||
-      !make_map_f32(&mdq, p.dq_acc, D, p.rows, p.heads) ||
+      !make_map_f32(&mdq, p.dq_acc, D, p.rows, 2LL * p.heads) ||
       !make_map_cols(&mcols, p.cols, (long long)p.heads * p.nseq * p.S_pad))
     return FA_ERR_CUDA;
   if (dropout)
@@ -273,10 +293,17 @@ fa_status launch_bwd_main(const void* q, const void* k, const void* v, const voi
                 : launch_bwd_main_t<D, BF16, false, false>(mq, mk, mv, mdo, mdq, mcols, p, st);
 }
 
+// det: bwd_main ran deterministic (two accumulators to add)
 template <bool BF16>
-fa_status launch_bwd_post(void* dq, const fa::BwdParams& p, int D, cudaStream_t st) {
+fa_status launch_bwd_post(void* dq, const fa::BwdParams& p, int D, cudaStream_t st, bool det) {
   const long long n8 = (long long)p.heads * p.rows * D / 8;
-  fa::bwd_post_kernel<BF16><<<sm_count() * 8, 256, 0, st>>>(p.dq_acc, static_cast<uint16_t*>(dq), n8, p.scale);
+  // 8 CTAs of 256 threads per SM, all resident at once
+  if (det)
+    fa::bwd_post_kernel<BF16, true><<<sm_count() * 8, 256, 0, st>>>(p.dq_acc, p.ticket + 1,
+                                                                     static_cast<uint16_t*>(dq), n8, p.scale);
+  else
+    fa::bwd_post_kernel<BF16, false><<<sm_count() * 8, 256, 0, st>>>(p.dq_acc, p.ticket + 1,
+                                                                      static_cast<uint16_t*>(dq), n8, p.scale);
   g_launches.fetch_add(1);
   return from_cuda(cudaGetLastError());
 }
@@ -299,7 +326,8 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* o, co
     c = bf16 ? launch_bwd_main<128, true>(q, k, v, dO, p, causal, varlen, dropout, st)
              : launch_bwd_main<128, false>(q, k, v, dO, p, causal, varlen, dropout, st);
   if (c != FA_OK) return c;
-  return bf16 ? launch_bwd_post<true>(dq, p, D, st) : launch_bwd_post<false>(dq, p, D, st);
+  return bf16 ? launch_bwd_post<true>(dq, p, D, st, p.deterministic != 0)
+              : launch_bwd_post<false>(dq, p, D, st, p.deterministic != 0);
 }
 
 // shared checks of the backward entry points: sizes, dtype, workspace
@@ -577,8 +605,8 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* d
                        : launch_bwd_main<128, false>(q, k, v, dO, p, cz, false, false, st);
 }
 
-fa_status fa_bwd_finish(void* dq, int B, int H, int S, int D, float scale, fa_dtype dt, void* workspace,
-                        size_t workspace_bytes, void* stream) {
+fa_status fa_bwd_finish(void* dq, int B, int H, int S, int D, float scale, fa_dtype dt, int deterministic,
+                        void* workspace, size_t workspace_bytes, void* stream) {
   fa_status c = bwd_common_checks(B, H, S, D, dt, workspace, workspace_bytes);
   if (c != FA_OK) return c;
   if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
@@ -587,7 +615,8 @@ fa_status fa_bwd_finish(void* dq, int B, int H, int S, int D, float scale, fa_dt
   const fa::BwdParams p =
       bwd_params(B * H, 1, S, S, nullptr, D, scale, 0, static_cast<uint8_t*>(workspace), nullptr, nullptr);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return dt == FA_BF16 ? launch_bwd_post<true>(dq, p, D, st) : launch_bwd_post<false>(dq, p, D, st);
+  return dt == FA_BF16 ? launch_bwd_post<true>(dq, p, D, st, deterministic != 0)
+                       : launch_bwd_post<false>(dq, p, D, st, deterministic != 0);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
@@ -603,7 +632,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   c = fa_bwd_main(q, k, v, dO, dk, dv, B, H, S, D, scale, causal, dt, deterministic, workspace, workspace_bytes,
                   stream);
   if (c != FA_OK) return c;
-  return fa_bwd_finish(dq, B, H, S, D, scale, dt, workspace, workspace_bytes, stream);
+  return fa_bwd_finish(dq, B, H, S, D, scale, dt, deterministic, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S,
@@ -803,7 +832,7 @@ fa_status fa_check_device_error(void* stream) {
   if (code == 0) return FA_OK;
   const uint32_t zero = 0;
   if (cudaMemcpyToSymbol(fa::g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
-  return FA_ERR_TIMEOUT;
+  return code == fa::DEV_ERR_ARG ? FA_ERR_INVALID_ARG : FA_ERR_TIMEOUT;
 }
 
 uint64_t fa_launch_count(void) { return g_launches.load(); }

@@ -57,14 +57,16 @@
 //                          a per-warp 128-byte-swizzled staging buffer and add
 //                          it to the fp32 accumulator with TMA bulk reductions
 //                          (cp.reduce.async.bulk.tensor .add); under
-//                          deterministic mode the key tiles take turns to
-//                          issue those reductions for tile i, from the highest
-//                          j down (the order in which they reach tile i), and
-//                          the units are numbered so that every key tile is
-//                          claimed after the one whose turn precedes it: that
-//                          one is always held by a running CTA, whatever order
-//                          the hardware starts CTAs in.
-//   bwd_post  dQ = scale * accumulator, rounded to the input dtype.
+//                          deterministic mode even and odd key tiles add into
+//                          two accumulators, and in each the key tiles take
+//                          turns for tile i, from the highest j down (the
+//                          order in which they reach tile i); the units are
+//                          numbered so that every key tile is claimed after
+//                          the one whose turn precedes it: that one is always
+//                          held by a running CTA, whatever order the hardware
+//                          starts CTAs in.
+//   bwd_post  dQ = scale * accumulator (+ the second one after a deterministic
+//             bwd_main), rounded to the input dtype.
 // Causal: key tile j only meets query tiles i >= j; only the diagonal tile
 // is masked element-wise.  Packed batches ([H, T, D], cu_seqlens): every
 // sequence is its own problem with tiles counted from its first token; keys
@@ -86,12 +88,14 @@ namespace fa {
 struct BwdParams {
   void* dk;                // [heads, rows, D]
   void* dv;                // [heads, rows, D]
-  float* dq_acc;           // [heads, rows, D] fp32
+  float* dq_acc;           // [2, heads, rows, D] fp32: the accumulator, then the second one of
+                           //   deterministic mode (odd key tiles)
   uint16_t* cols;          // [heads, nseq, S_pad, 16] bf16 per-query rows (written by bwd_pre):
                            //   0-8: -LSE*log2(e) in three parts (part k % 3 in column k),
                            //   9-11: -D_i in three parts, 12-15: 0; padding rows -1e30 and 0
-  uint32_t* sem;           // [heads, nseq, n_q] ordering counters (deterministic mode)
-  uint32_t* ticket;        // next unit to claim (zeroed by bwd_pre)
+  uint32_t* sem;           // [heads, nseq, n_q, 2] ordering counters (deterministic mode, per chain)
+  uint32_t* ticket;        // next unit to claim (zeroed by bwd_pre); ticket[1]: nonzero once a
+                           //   deterministic bwd_main has filled the second accumulator
   const int* cu_seqlens;   // packed batch only: device int32 [nseq + 1]
   int heads;               // dense: B*H, packed: H
   int S;                   // dense: S, packed: max_seqlen
@@ -119,7 +123,7 @@ struct BwdCfg {
   static constexpr uint32_t ONES_OFF = CT_OFF + 2 * 4096;         // the two constant key-side rows (128 x 32 B)
   static constexpr uint32_t BAR_OFF = ONES_OFF + 2 * 4096;
   // kv_full kv_empty q_full[2] q_empty[2] do_full do_empty s_full dp_full
-  // p_full dp_taken ds_full dq_full dq_empty dkv_full drain dq_done
+  // p_full dp_taken ds_full dq_full dq_empty dkv_full drain (one unused)
   // unit_full[2] unit_empty[2]
   static constexpr int NBAR = 22;
   // then the TMEM address and the two-slot unit ring
@@ -134,7 +138,7 @@ enum : uint32_t {
   BWD_SITE_PROD = 0x200, BWD_SITE_KV = 0x201, BWD_SITE_Q = 0x202, BWD_SITE_DO = 0x203, BWD_SITE_P = 0x204,
   BWD_SITE_DS = 0x205, BWD_SITE_DQE = 0x206, BWD_SITE_S = 0x207, BWD_SITE_DP = 0x208, BWD_SITE_DQF = 0x209,
   BWD_SITE_DKV = 0x20a, BWD_SITE_SEM = 0x20b, BWD_SITE_DRAIN = 0x20c, BWD_SITE_STAT = 0x20d, BWD_SITE_UNIT = 0x20e,
-  BWD_SITE_TAKEN = 0x20f
+  BWD_SITE_TAKEN = 0x20f, BWD_SITE_POST = 0x210
 };
 
 // One work unit: key/value tile j of one (sequence, head) slice, which meets
@@ -251,21 +255,42 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict
   const long long n4 = (long long)p.heads * p.rows * D / 4;
   float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
   for (long long i = gtid; i < n4; i += nthreads) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  const long long ns = (long long)p.heads * p.nseq * p.n_q;
+  const long long ns = (long long)p.heads * p.nseq * p.n_q * 2;
   for (long long i = gtid; i < ns; i += nthreads) p.sem[i] = 0u;
-  if (gtid == 0) *p.ticket = 0u;
+  if (gtid == 0) {
+    p.ticket[0] = 0u;
+    p.ticket[1] = 0u;
+  }
 }
 
 // ---------------------------------------------------------------------------
 // bwd_post: dQ = scale * accumulator, rounded to nearest in the input dtype.
+// TWO (deterministic bwd_main): the odd key tiles' sums sit in a second
+// accumulator n8 * 8 floats further on, added to the first in this order.
+// Separate instances, each held to the 32 registers that let the launch's 8
+// CTAs per SM all be resident at once.
+// bwd_main left its own word in *det (nonzero: deterministic); one thread
+// compares it with TWO, with the load issued before the loop so that it
+// costs no time, and records DEV_ERR_ARG when they disagree (the result then
+// misses the odd key tiles, or adds a stale second accumulator).
 // ---------------------------------------------------------------------------
-template <bool BF16>
-__global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, uint16_t* __restrict__ dq,
-                                                       long long n8, float scale) {
+template <bool BF16, bool TWO>
+__global__ void __launch_bounds__(256, 8) bwd_post_kernel(const float* __restrict__ acc, const uint32_t* __restrict__ det,
+                                                       uint16_t* __restrict__ dq, long long n8, float scale) {
+  const bool checker = blockIdx.x == 0 && threadIdx.x == 0;
+  uint32_t left = 0;
+  if (checker) left = __ldcg(det);
+  const float* acc2 = acc + n8 * 8;
   const long long nthreads = (long long)gridDim.x * blockDim.x;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += nthreads) {
-    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
-    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+    float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    if constexpr (TWO) {
+      const float4 a2 = reinterpret_cast<const float4*>(acc2)[2 * i];
+      const float4 b2 = reinterpret_cast<const float4*>(acc2)[2 * i + 1];
+      a = make_float4(a.x + a2.x, a.y + a2.y, a.z + a2.z, a.w + a2.w);
+      b = make_float4(b.x + b2.x, b.y + b2.y, b.z + b2.z, b.w + b2.w);
+    }
     uint4 r;
     r.x = pack2<BF16>(a.x * scale, a.y * scale);
     r.y = pack2<BF16>(a.z * scale, a.w * scale);
@@ -273,6 +298,7 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
     r.w = pack2<BF16>(b.z * scale, b.w * scale);
     reinterpret_cast<uint4*>(dq)[i] = r;
   }
+  if (checker && (left != 0u) != TWO) record_error(DEV_ERR_ARG, BWD_SITE_POST);
 }
 
 // fp32 tile in shared memory added element-wise into global memory by the
@@ -296,6 +322,9 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -303,7 +332,9 @@ __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
 // ---------------------------------------------------------------------------
 // bwd_main
 // ---------------------------------------------------------------------------
-template <int D, bool BF16, bool CAUSAL, bool VARLEN, bool DROPOUT = false>
+// DET: deterministic mode (p.deterministic), a separate instance so that the
+// atomic mode's dQ warps carry none of its ordering state.
+template <int D, bool BF16, bool CAUSAL, bool VARLEN, bool DROPOUT = false, bool DET = false>
 __global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -328,7 +359,6 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* dq_empty = bars + 14;  // dQ(g) read out of X(g) (128 dQ threads)
   uint64_t* dkv_full = bars + 15;  // the unit's dV and dK are final
   uint64_t* drain = bars + 16;
-  uint64_t* dq_done = bars + 17;   // deterministic mode: this tile's dQ reductions performed (128 dQ threads)
   uint64_t* unit_full = bars + 18;   // [2] a claimed unit number is in the ring
   uint64_t* unit_empty = bars + 20;  // [2] every role has read it (one lane of each of 13 warps)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBAR);
@@ -358,7 +388,6 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(dq_empty, 128);
     mbar_init(dkv_full, 1);
     mbar_init(drain, 1);
-    mbar_init(dq_done, 128);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -821,13 +850,20 @@ __global__ void __launch_bounds__(512, 1)
   } else {
     regs_inc<RQ>();
     // ------------------------------------------------------------ dQ (one thread per query row)
-    const int c = threadIdx.x - 384;                 // query row within the tile = TMEM lane
     const int wq = warp - 12;                        // this warp's 32 rows: 32*wq ..
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     uint8_t* stg = smem + C::STG_OFF + wq * 4096;    // 32 rows x 128 B, 128-B swizzled
     if (lane == 0) tma_prefetch_desc(&tm_dq);
     uint32_t g = 0;  // query steps so far
     bool ok = true;
+    // deterministic mode: the chain counter this warp still owes its count
+    // to (the last step's)
+    uint32_t* pend_new = nullptr;
+    auto count_in = [&](uint32_t* sem) {  // lane 0, once that step's reductions have been performed
+      fence_proxy_async_global();
+      __threadfence();
+      red_release_gpu_add(sem, 1u);
+    };
     for (int k = 0; ok; ++k) {
       int u;
       if (!(ok = next_unit(k, u)) || u < 0) break;
@@ -850,7 +886,7 @@ __global__ void __launch_bounds__(512, 1)
         BWD_TRACE(qw, 2400 + 3 * g + 1);
         // This tile's fp32 partial: TMEM -> per-warp swizzled staging -> TMA bulk
         // reduce-add into the accumulator, 32 columns at a time.
-        auto reduce_partial = [&]() {
+        auto reduce_partial = [&](int hc) {  // hc: the head coordinate in the accumulator map
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
             if (lane == 0) bulk_wait_read0();  // the previous reduction has read the buffer
@@ -862,53 +898,64 @@ __global__ void __launch_bounds__(512, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_reduce_add_3d(&tm_dq, stg, 32 * cc, x.row_base + 128 * i + 32 * wq, x.head);
+              tma_reduce_add_3d(&tm_dq, stg, 32 * cc, x.row_base + 128 * i + 32 * wq, hc);
               bulk_commit();
             }
           }
         };
-        if (!p.deterministic) {
-          reduce_partial();
+        if constexpr (!DET) {
+          reduce_partial(x.head);
           BWD_TRACE(qw, 2400 + 3 * g + 2);
         } else {
-          // Key tiles add into query tile i in a fixed order: one poller per
-          // warp waits for our turn, the partial goes in with the same bulk
-          // reductions, and the turn passes on only once they have been
-          // performed, so every element sees its additions in one fixed order.
-          uint32_t* sem = p.sem + ((size_t)x.head * p.nseq + x.seq) * p.n_q + i;
-          // key tiles add into query tile i from the highest down: j = i first
-          // under the causal mask (j = n_q - 1 without it), then j - 1, ...
-          const uint32_t turn = (uint32_t)((CAUSAL ? i : x.n_q - 1) - x.j);
-          bool mine = true;
+          // Key tiles add into query tile i in a fixed order, in two chains:
+          // even j into the first accumulator, odd j into the second, each
+          // from its highest j down (j = i or i - 1 first under the causal
+          // mask, j = n_q - 1 or n_q - 2 without it).  A chain's counter for
+          // tile i counts the dQ warps (four per key tile) whose reductions
+          // into it have been performed: a warp waits until all four warps of
+          // every earlier key tile of the chain are in, adds its partial with
+          // the same bulk reductions, and adds its own one only once those
+          // have been performed, so every element sees its additions in one
+          // fixed order.  The count is added one step later, after the next
+          // partial has been drained, or at once after a unit's last tile; the
+          // predecessor in the chain, key tile j + 2, reached tile i two steps
+          // before us under the causal mask, which leaves that hand-over a
+          // step of time.  (Counting two steps later, so that the completion
+          // wait leaves the warp's loop, measured slower.)
+          if (pend_new && lane == 0) {
+            bulk_wait0();
+            count_in(pend_new);
+          }
+          pend_new = nullptr;
+          const int chain = x.j & 1;
+          const int top = CAUSAL ? i : x.n_q - 1;
+          const uint32_t turn = (uint32_t)((top - ((top - chain) & 1) - x.j) >> 1);
+          uint32_t* sem = p.sem + (((size_t)x.head * p.nseq + x.seq) * p.n_q + i) * 2 + chain;
           if (lane == 0) {
-            if (ld_acquire_gpu(sem) != turn) {
+            if (ld_acquire_gpu(sem) < 4u * turn) {
               const uint64_t t0 = global_ns();
-              while (ld_acquire_gpu(sem) != turn) {
+              while (ld_acquire_gpu(sem) < 4u * turn) {
                 if (global_ns() - t0 > kWaitLimitNs) {
+                  // reported; go on so that the later key tiles are not held up too
                   record_error(DEV_ERR_TIMEOUT, BWD_SITE_SEM);
-                  mine = false;
                   break;
                 }
               }
             }
             fence_proxy_async_global();  // our reductions come after the acquire
           }
-          mine = __shfl_sync(0xffffffffu, mine, 0);
-          if (mine) {
-            reduce_partial();
+          __syncwarp();
+          BWD_TRACE(qw, 2400 + 3 * g + 2);
+          reduce_partial(x.head + chain * p.heads);
+          pend_new = sem;
+          if (st == x.n_steps - 1) {  // a unit's last tile: count it in now
             if (lane == 0) {
-              bulk_wait0();  // this warp's reductions have been performed
-              fence_proxy_async_global();
+              bulk_wait0();
+              count_in(pend_new);
             }
+            pend_new = nullptr;
           }
           __syncwarp();
-          mbar_arrive(dq_done);
-          if (c == 0) {
-            if (mbar_wait(dq_done, g & 1, BWD_SITE_SEM) && mine) {
-              __threadfence();
-              st_release_gpu(sem, turn + 1);
-            }
-          }
         }
       }
     }

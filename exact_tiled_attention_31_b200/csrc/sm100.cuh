@@ -12,10 +12,11 @@
 namespace fa {
 
 // ---------------------------------------------------------------------------
-// Device error word.  A wait that gives up records why and where; the host
-// reads it with fa_check_device_error().
+// Device error word.  A wait that gives up, or a check that fails, records
+// why and where; the host reads it with fa_check_device_error().
+// DEV_ERR_ARG: calls that had to agree did not (see bwd_post).
 // ---------------------------------------------------------------------------
-enum : uint32_t { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1 };
+enum : uint32_t { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1, DEV_ERR_ARG = 2 };
 
 // Defined here: each shared library is built from a single translation unit.
 __device__ uint32_t g_dev_error = 0;   // first error code (0 = none)

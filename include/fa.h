@@ -94,11 +94,12 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
                         int H, int D, float scale, int causal, fa_dtype dt, void* stream);
 
 /*
- * Bytes of device scratch that fa_bwd needs for these sizes: an fp32 dQ
- * accumulator [B, H, S, D], one 32-byte row per query (LSE and the row term
+ * Bytes of device scratch that fa_bwd needs for these sizes: two fp32 dQ
+ * accumulators [B, H, S, D] (the second holds the odd key tiles' sums in
+ * deterministic mode), one 32-byte row per query (LSE and the row term
  * D_i = dO_i . O_i, as bf16 parts, rows padded to multiples of 128), the
- * ordering counters of deterministic mode and the work counter of the
- * backward's persistent grid, each 256-byte aligned.
+ * ordering counters of deterministic mode (two per query tile) and the work
+ * counter of the backward's persistent grid, each 256-byte aligned.
  * Returns 0 for unsupported sizes.
  * This is the first half of the two-phase call of the operator in
  * "ops-transformer里的FlashAttention", "ops-transformer里的完整算子": a size
@@ -116,10 +117,12 @@ size_t fa_bwd_workspace_size(int B, int H, int S, int D);
  * deterministic = 0: dQ partial sums from different key tiles are added with
  *   fp32 reductions (TMA bulk reduce-adds) in whatever order the key tiles
  *   reach them, so dq may differ in the last bits from run to run.
- * deterministic = 1: the key tiles of one query tile add their dQ partials in
- *   increasing key-tile order, so repeated calls with the same inputs, sizes
- *   and GPU give bit-identical dq (the `deterministic` option of the
- *   operator config in "ops-transformer里的FlashAttention", "ops-transformer里的完整算子").
+ * deterministic = 1: the dQ partials of one query tile are added in a fixed
+ *   order: the even key tiles into one fp32 accumulator and the odd ones
+ *   into another, each from the highest key tile down, and the two sums are
+ *   added at the end, so repeated calls with the same inputs, sizes and GPU
+ *   give bit-identical dq (the `deterministic` option of the operator config
+ *   in "ops-transformer里的FlashAttention", "ops-transformer里的完整算子").
  * The gradients are those of L = sum(dO * O): dV = P^T dO, dS = P o (dP - D),
  * dQ = scale dS K, dK = scale dS^T Q, with P rebuilt from lse
  * ("Flash Attention 的算法设计原理", "核心机制"; the pages print no formulas, these
@@ -167,14 +170,21 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
  *                      its units from.
  *   fa_bwd_main        the tiled pass over key/value tiles: writes dk, dv
  *                      and accumulates unscaled dQ (fp32) in the workspace.
- *   fa_bwd_finish      dq = scale * accumulated dQ, rounded to the dtype.
+ *   fa_bwd_finish      dq = scale * accumulated dQ (the sum of both
+ *                      accumulators when deterministic), rounded to the
+ *                      dtype.  `deterministic` must be the value given to
+ *                      fa_bwd_main; the kernel compares it with the mark
+ *                      fa_bwd_main left in the workspace and, when they
+ *                      differ, records an argument error that
+ *                      fa_check_device_error() returns as FA_ERR_INVALID_ARG
+ *                      (dq is then wrong).
  */
 fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int S, int D,
                             fa_dtype dt, void* workspace, size_t workspace_bytes, void* stream);
 fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
                       int B, int H, int S, int D, float scale, int causal, fa_dtype dt, int deterministic,
                       void* workspace, size_t workspace_bytes, void* stream);
-fa_status fa_bwd_finish(void* dq, int B, int H, int S, int D, float scale, fa_dtype dt,
+fa_status fa_bwd_finish(void* dq, int B, int H, int S, int D, float scale, fa_dtype dt, int deterministic,
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
@@ -328,8 +338,10 @@ const char* fa_status_string(fa_status s);
 
 /*
  * Synchronises `stream`, then reads and clears the calling device's error
- * word.  Returns FA_OK, FA_ERR_TIMEOUT (a kernel gave up waiting) or
- * FA_ERR_CUDA (the synchronisation itself failed).  No page defines this
+ * word.  Returns FA_OK, FA_ERR_TIMEOUT (a kernel gave up waiting),
+ * FA_ERR_INVALID_ARG (fa_bwd_finish was told another deterministic mode
+ * than fa_bwd_main ran in) or FA_ERR_CUDA (the synchronisation itself
+ * failed).  No page defines this
  * call; it is the host side of the library's bounded-wait error handling.
  */
 fa_status fa_check_device_error(void* stream);

@@ -46,8 +46,8 @@ def test_workspace_size_formula(lib):
         return (x + 255) // 256 * 256
     for B, H, S, D in [(1, 32, 4096, 128), (2, 3, 17, 64), (4, 16, 8192, 128)]:
         heads, spad = B * H, (S + 127) // 128 * 128
-        # fp32 dQ accumulator, per-query rows, ordering counters, the work counter
-        expect = up(heads * S * D * 4) + up(heads * spad * 32) + up(heads * (spad // 128) * 4) + 256
+        # two fp32 dQ accumulators, per-query rows, ordering counters (two chains), the work counter
+        expect = up(2 * heads * S * D * 4) + up(heads * spad * 32) + up(heads * (spad // 128) * 2 * 4) + 256
         assert fa.fa_bwd_workspace_size(B, H, S, D) == expect
     assert fa.fa_bwd_workspace_size(1, 1, 16, 96) == 0
     assert fa.fa_bwd_workspace_size(0, 1, 16, 64) == 0
@@ -102,7 +102,7 @@ def test_bwd_varlen_workspace_and_argument_errors(lib):
         return (x + 255) // 256 * 256
     nseq, mx, T, H, D = 3, 300, 500, 4, 128
     spad = (mx + 127) // 128 * 128
-    expect = up(H * T * D * 4) + up(H * nseq * spad * 32) + up(H * nseq * (spad // 128) * 4) + 256
+    expect = up(2 * H * T * D * 4) + up(H * nseq * spad * 32) + up(H * nseq * (spad // 128) * 2 * 4) + 256
     assert fa.fa_bwd_varlen_workspace_size(nseq, mx, T, H, D) == expect
     assert fa.fa_bwd_varlen_workspace_size(nseq, mx, T, H, 96) == 0
     assert fa.fa_bwd_varlen_workspace_size(0, mx, T, H, D) == 0

@@ -133,7 +133,32 @@ def test_bwd_split_launches_equal_fa_bwd(cuda_device):
                                 st) == 0
     assert fa.fa_bwd_main(d["q"].data_ptr(), d["k"].data_ptr(), d["v"].data_ptr(), d["do"].data_ptr(), dk.data_ptr(),
                           dv.data_ptr(), B, H, S, D, 0.088, True, dt, True, ws.data_ptr(), nb, st) == 0
-    assert fa.fa_bwd_finish(dq.data_ptr(), B, H, S, D, 0.088, dt, ws.data_ptr(), nb, st) == 0
+    assert fa.fa_bwd_finish(dq.data_ptr(), B, H, S, D, 0.088, dt, True, ws.data_ptr(), nb, st) == 0
     fa.check_device_error()
     for a, b, name in zip((dq, dk, dv), ref, ("dQ", "dK", "dV")):
         assert torch.equal(a, b), name
+
+
+@pytest.mark.parametrize("det_main", [False, True])
+def test_bwd_split_mode_mismatch_is_reported(cuda_device, det_main):
+    """fa_bwd_finish told the other deterministic mode than fa_bwd_main ran
+    in records an argument error (read back as FA_ERR_INVALID_ARG, which also
+    clears it); the same calls with matching modes record none."""
+    B, H, S, D = 1, 2, 300, 64
+    t = inputs.make_dense(B, H, S, D, "bf16", seed=9, with_do=True)
+    d = to_dev(t, cuda_device)
+    o, lse = fa.forward(d["q"], d["k"], d["v"], False, 0.125)
+    nb = fa.fa_bwd_workspace_size(B, H, S, D)
+    ws = torch.empty(nb, dtype=torch.uint8, device=cuda_device)
+    dq, dk, dv = (torch.empty_like(d["q"]) for _ in range(3))
+    st = torch.cuda.current_stream().cuda_stream
+    dt = fa.api.FA_BF16
+    fa.check_device_error()
+    for det_finish, want in ((not det_main, fa.api.FA_ERR_INVALID_ARG), (det_main, fa.api.FA_OK)):
+        assert fa.fa_bwd_preprocess(o.data_ptr(), d["do"].data_ptr(), lse.data_ptr(), B, H, S, D, dt, ws.data_ptr(),
+                                    nb, st) == 0
+        assert fa.fa_bwd_main(d["q"].data_ptr(), d["k"].data_ptr(), d["v"].data_ptr(), d["do"].data_ptr(),
+                              dk.data_ptr(), dv.data_ptr(), B, H, S, D, 0.125, False, dt, det_main, ws.data_ptr(), nb,
+                              st) == 0
+        assert fa.fa_bwd_finish(dq.data_ptr(), B, H, S, D, 0.125, dt, det_finish, ws.data_ptr(), nb, st) == 0
+        assert fa.fa_check_device_error(st) == want
