@@ -71,7 +71,7 @@ struct DecCfg {
   static_assert((WARPS + 1) * SCRATCH * 4 <= WARPS * WARP_BYTES, "merge scratch fits in the tile buffers");
 };
 
-enum : uint32_t { DEC_SITE_KV = 0x300, DEC_SITE_DRAIN = 0x301 };
+enum : uint32_t { DEC_SITE_KV = 0x300, DEC_SITE_DRAIN = 0x301, DEC_SITE_MERGE = 0x302 };
 
 // byte offset of (row, 8-column chunk c8 of D / 8) in a K or V tile
 template <int D>
@@ -548,11 +548,20 @@ __global__ void __launch_bounds__(128, 1)
 // exp(LSE_s), O = sum exp(LSE_s - LSE) O_s.  One block of D threads per row.
 // Launched as a programmatic dependent of the split or balanced kernel: its
 // blocks may be resident before that kernel ends and wait here for its
-// results.
+// results.  Every load whose address is known is issued before the first
+// result is needed: thread d's column of the first kPrefetch parts, and the
+// parts' LSEs spread over the threads, so a row costs about one memory
+// latency instead of one per part.  A row has at most kMergeMax parts (the
+// host allows at most 1024 splits and 1024 balanced-mode CTAs).
+constexpr int kMergeMax = 1024, kPrefetch = 16;
+
 template <int D, bool BF16>
 __global__ void __launch_bounds__(D) decode_merge_kernel(const DecParams p) {
+  __shared__ float w_s[kMergeMax];  // the parts' LSEs, then their weights exp(LSE_s - max)
+  __shared__ float red[D / 32];
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const size_t row = blockIdx.x;  // b * Hq + h
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   // the row's parts: n of them, part s at index part_at(s) of lse_part (and
   // of o_part in rows of D)
   int n;
@@ -576,21 +585,55 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecParams p) {
     rest0 = first + p.group;
     rest_stride = p.group;
   }
-  auto part_at = [&](int s) { return s == 0 ? first : rest0 + (size_t)(s - 1) * rest_stride; };
-  float mx = -INFINITY;
-  for (int s = 0; s < n; ++s) mx = fmaxf(mx, p.lse_part[part_at(s)]);
-  float tot = 0.f, acc = 0.f;
-  for (int s = 0; s < n; ++s) {
-    const size_t idx = part_at(s);
-    const float w = mx == -INFINITY ? 0.f : __expf(p.lse_part[idx] - mx);
-    tot += w;
-    acc += w * p.o_part[idx * D + threadIdx.x];
+  if (n > kMergeMax) {  // excluded by the host's limits
+    if (t == 0) record_error(DEV_ERR_ARG, DEC_SITE_MERGE);
+    return;
   }
+  auto part_at = [&](int s) { return s == 0 ? first : rest0 + (size_t)(s - 1) * rest_stride; };
+  float ov[kPrefetch];
+#pragma unroll
+  for (int s = 0; s < kPrefetch; ++s) ov[s] = s < n ? p.o_part[part_at(s) * D + t] : 0.f;
+  float mx = -INFINITY;
+  for (int s = t; s < n; s += D) {
+    const float l = p.lse_part[part_at(s)];
+    w_s[s] = l;
+    mx = fmaxf(mx, l);
+  }
+  // block maximum
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  mx = red[0];
+#pragma unroll
+  for (int w = 1; w < D / 32; ++w) mx = fmaxf(mx, red[w]);
+  __syncthreads();  // red is reused below
+  // weights (all zero when every part is empty) and their sum
+  float tot = 0.f;
+  for (int s = t; s < n; s += D) {
+    const float w = mx == -INFINITY ? 0.f : __expf(w_s[s] - mx);
+    w_s[s] = w;
+    tot += w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  if (lane == 0) red[warp] = tot;
+  __syncthreads();  // w_s and red are complete
+  tot = red[0];
+#pragma unroll
+  for (int w = 1; w < D / 32; ++w) tot += red[w];
+  // O column t, parts added in order
+  float acc = 0.f;
+#pragma unroll
+  for (int s = 0; s < kPrefetch; ++s)
+    if (s < n) acc += w_s[s] * ov[s];
+#pragma unroll 8
+  for (int s = kPrefetch; s < n; ++s) acc += w_s[s] * p.o_part[part_at(s) * D + t];
   const float o = tot > 0.f ? acc / tot : 0.f;
-  uint16_t* dst = static_cast<uint16_t*>(p.o) + row * D + threadIdx.x;
+  uint16_t* dst = static_cast<uint16_t*>(p.o) + row * D + t;
   const uint32_t pk = pack2<BF16>(o, 0.f);
   *dst = (uint16_t)(pk & 0xffffu);
-  if (threadIdx.x == 0) p.lse[row] = tot > 0.f ? mx + __logf(tot) : -INFINITY;
+  if (t == 0) p.lse[row] = tot > 0.f ? mx + __logf(tot) : -INFINITY;
 }
 
 }  // namespace fa
