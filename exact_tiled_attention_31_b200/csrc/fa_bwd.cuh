@@ -43,6 +43,9 @@
 //                          so the next step's exponentials start while dK,
 //                          dQ and the next dP^T are on the tensor core.
 //                          dV [256,256+D), dK [256+D,256+2D).
+//               warp 2     deterministic mode only: adds the dQ warps'
+//                          counts to the ordering counters (one gpu-scope
+//                          release per step, off the dQ warps' path).
 //               warps 4-11 one thread per key row and half of the query
 //                          columns (warps 4-7 queries 0-63, 8-11 queries
 //                          64-127).  P phase: P^T = exp2(S'^T*scale*log2e)
@@ -124,10 +127,11 @@ struct BwdCfg {
   static constexpr uint32_t BAR_OFF = ONES_OFF + 2 * 4096;
   // kv_full kv_empty q_full[2] q_empty[2] do_full do_empty s_full dp_full
   // p_full dp_taken ds_full dq_full dq_empty dkv_full drain (one unused)
-  // unit_full[2] unit_empty[2]
-  static constexpr int NBAR = 22;
-  // then the TMEM address and the two-slot unit ring
-  static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
+  // unit_full[2] unit_empty[2] rel_full[2] rel_empty[2]
+  static constexpr int NBAR = 26;
+  // then the TMEM address, the two-slot unit ring, and the two-slot ring of
+  // counters the release warp adds to
+  static constexpr uint32_t SMEM = BAR_OFF + NBAR * 8 + 32 + 1024;
   static constexpr uint32_t TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
 };
 
@@ -138,7 +142,7 @@ enum : uint32_t {
   BWD_SITE_PROD = 0x200, BWD_SITE_KV = 0x201, BWD_SITE_Q = 0x202, BWD_SITE_DO = 0x203, BWD_SITE_P = 0x204,
   BWD_SITE_DS = 0x205, BWD_SITE_DQE = 0x206, BWD_SITE_S = 0x207, BWD_SITE_DP = 0x208, BWD_SITE_DQF = 0x209,
   BWD_SITE_DKV = 0x20a, BWD_SITE_SEM = 0x20b, BWD_SITE_DRAIN = 0x20c, BWD_SITE_STAT = 0x20d, BWD_SITE_UNIT = 0x20e,
-  BWD_SITE_TAKEN = 0x20f, BWD_SITE_POST = 0x210
+  BWD_SITE_TAKEN = 0x20f, BWD_SITE_POST = 0x210, BWD_SITE_REL = 0x211
 };
 
 // One work unit: key/value tile j of one (sequence, head) slice, which meets
@@ -361,8 +365,12 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* drain = bars + 16;
   uint64_t* unit_full = bars + 18;   // [2] a claimed unit number is in the ring
   uint64_t* unit_empty = bars + 20;  // [2] every role has read it (one lane of each of 13 warps)
+  uint64_t* rel_full = bars + 22;    // [2] deterministic mode: the four dQ warps' reductions of a
+                                     //   step are performed and its counter is in rel_sem
+  uint64_t* rel_empty = bars + 24;   // [2] the release warp has taken the counter
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* unit_ring = reinterpret_cast<volatile int*>(tmem_holder + 1);  // [2]
+  uint32_t* volatile* rel_sem = reinterpret_cast<uint32_t* volatile*>(tmem_holder + 4);  // [2]
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
@@ -376,6 +384,8 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&q_empty[i], 1);
       mbar_init(&unit_full[i], 1);
       mbar_init(&unit_empty[i], 13);
+      mbar_init(&rel_full[i], 4);
+      mbar_init(&rel_empty[i], 1);
     }
     mbar_init(do_full, 1);
     mbar_init(do_empty, 1);
@@ -613,6 +623,26 @@ __global__ void __launch_bounds__(512, 1)
     }
     mma_commit_e(drain, e);
     mbar_wait(drain, 0, BWD_SITE_DRAIN);
+    __syncwarp();
+  } else if (DET && warp == 2) {
+    // ------------------------------------------------------------ release
+    // Deterministic mode: adds each step's four dQ-warp counts to its chain
+    // counter with one gpu-scope release, which takes ~1100 clk that the dQ
+    // warps would otherwise wait out every step.  Each dQ warp's lane 0 has
+    // waited for its reductions and fenced them against the generic proxy
+    // before arriving on rel_full (a CTA-scope release); the wait here
+    // acquires that, and the release below passes it on to the next key
+    // tile's acquire.  A null counter ends the loop.
+    if (lane == 0) {
+      for (uint32_t h = 0;; ++h) {
+        const int slot = h & 1;
+        if (!mbar_wait(&rel_full[slot], (h >> 1) & 1, BWD_SITE_REL)) break;
+        uint32_t* sem = rel_sem[slot];
+        mbar_arrive(&rel_empty[slot]);
+        if (!sem) break;
+        red_release_gpu_add(sem, 4u);
+      }
+    }
     __syncwarp();
   }
   } else if (warp < 12) {
@@ -857,12 +887,18 @@ __global__ void __launch_bounds__(512, 1)
     uint32_t g = 0;  // query steps so far
     bool ok = true;
     // deterministic mode: the chain counter this warp still owes its count
-    // to (the last step's)
+    // to (the last step's), and the posts made to the release warp
     uint32_t* pend_new = nullptr;
-    auto count_in = [&](uint32_t* sem) {  // lane 0, once that step's reductions have been performed
+    uint32_t posts = 0;
+    // lane 0, once this warp's reductions of that step have been performed:
+    // hand the counter to the release warp (null: no more steps)
+    auto count_in = [&](uint32_t* sem) {
+      const int slot = posts & 1;
+      if (posts >= 2 && !mbar_wait(&rel_empty[slot], ((posts >> 1) - 1) & 1, BWD_SITE_REL)) return;
+      if (warp == 12) rel_sem[slot] = sem;
       fence_proxy_async_global();
-      __threadfence();
-      red_release_gpu_add(sem, 1u);
+      mbar_arrive(&rel_full[slot]);
+      ++posts;
     };
     for (int k = 0; ok; ++k) {
       int u;
@@ -914,14 +950,15 @@ __global__ void __launch_bounds__(512, 1)
           // tile i counts the dQ warps (four per key tile) whose reductions
           // into it have been performed: a warp waits until all four warps of
           // every earlier key tile of the chain are in, adds its partial with
-          // the same bulk reductions, and adds its own one only once those
-          // have been performed, so every element sees its additions in one
-          // fixed order.  The count is added one step later, after the next
-          // partial has been drained, or at once after a unit's last tile; the
-          // predecessor in the chain, key tile j + 2, reached tile i two steps
-          // before us under the causal mask, which leaves that hand-over a
-          // step of time.  (Counting two steps later, so that the completion
-          // wait leaves the warp's loop, measured slower.)
+          // the same bulk reductions, and is counted only once those have
+          // been performed (the release warp adds the four warps' counts), so
+          // every element sees its additions in one fixed order.  The count
+          // is posted one step later, after the next partial has been
+          // drained, when the reductions have mostly completed, or at once
+          // after a unit's last tile; the predecessor in the chain, key tile
+          // j + 2, reached tile i two steps before us under the causal mask,
+          // which leaves that hand-over a step of time.  (Three chains with
+          // the count two steps later measured slower.)
           if (pend_new && lane == 0) {
             bulk_wait0();
             count_in(pend_new);
@@ -959,7 +996,10 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
     }
-    if (lane == 0) bulk_wait0();  // every reduction issued by this warp has completed
+    if (lane == 0) {
+      bulk_wait0();  // every reduction issued by this warp has completed
+      if constexpr (DET) count_in(nullptr);  // the release warp may stop
+    }
     __syncwarp();
   }
 
