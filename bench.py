@@ -63,12 +63,12 @@ def flops(w):
 # profiles/, with a digest of the kernel sources (code only) they were taken on.
 # Reported only while that code is unchanged (otherwise null: the counters are stale).
 NCU_TRAFFIC = {
-    "bwd_main": (290_289_289, "38e7e701e3699f87901d35c1bedd4d82be544e1b4d3fe93cc960ed01b7519252",
+    "bwd_main": (289_130_957, "015da12a81d87b63e77598732a9fcbca3eca84d1bbd4ee8eb74bb88f2f4bc66f",
                  ("fa_bwd.cuh", "sm100.cuh")),
-    "fwd": (151_981_073, "60d40782546f254928a296b48e46227a32b0386512a60093b94047a7f3b88867",
+    "fwd": (149_943_885, "60d40782546f254928a296b48e46227a32b0386512a60093b94047a7f3b88867",
             ("fa_fwd.cuh", "sm100.cuh")),
     # decode split kernel, B8 Hq32 Hkv8 L8192 D128 bf16, 2 splits merged in-kernel (mean of 13 launches)
-    "decode": (269_364_303, "94a39f624c60de04b4b8e9db037b53a1ad44dedd3f04b6f1889f98ec0dc51c8a",
+    "decode": (268_978_708, "4696a7ff08d2327e8bf9a19eb0d9726cd3c9d323b54f6fb50c07502f9a1c391b",
                ("fa_decode.cuh", "sm100.cuh")),
 }
 

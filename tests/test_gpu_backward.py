@@ -102,6 +102,26 @@ def test_bwd_deterministic_is_bitwise_repeatable(cuda_device):
         check_grad(b, a, f"{name} atomic vs ordered")
 
 
+@pytest.mark.parametrize("S", [1, 17, 129, 255, 383])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_deterministic_on_dirty_workspace_matches_oracle(cuda_device, S, D, causal):
+    """Deterministic mode on a workspace full of 0x7F bytes (3.4e38 as fp32),
+    ragged lengths, one tile and several: both dQ accumulators must be
+    cleared inside the call (the second one holds the odd key tiles, and no
+    key tile at all reaches it for query tile 0 under the causal mask), so
+    no byte from before the call may reach dQ."""
+    B, H = 2, 2
+    t = inputs.make_dense(B, H, S, D, "bf16", seed=S * D + causal, with_do=True)
+    d = to_dev(t, cuda_device)
+    scale = 1 / math.sqrt(D)
+    o, lse = fa.forward(d["q"], d["k"], d["v"], causal, scale)
+    ws = torch.full((fa.fa_bwd_workspace_size(B, H, S, D),), 0x7F, dtype=torch.uint8, device=cuda_device)
+    g = fa.backward(d["q"], d["k"], d["v"], o, d["do"], lse, causal, scale, deterministic=True, workspace=ws)
+    fa.check_device_error()
+    _check_all(t, causal, scale, (o, lse, *g), what=f"deterministic S={S} D={D} causal={causal}")
+
+
 def test_bwd_workspace_reuse_and_dirty(cuda_device):
     """The workspace may hold anything on entry (it is cleared inside)."""
     t = inputs.make_dense(1, 2, 640, 64, "fp16", seed=4, with_do=True)
