@@ -28,7 +28,9 @@
 //               12-19 tile 1; within a tile, warps 4k..4k+3 take keys 0-63
 //               and the next four keys 64-127 of the same 128 rows (TMEM
 //               lanes).  The two halves of a row swap their partial maxima
-//               through shared memory, then exponentiate in the log2 domain
+//               through shared memory (one barrier per 32 rows: the two
+//               warps of those rows and the correction warp that rescales
+//               them), then exponentiate in the log2 domain
 //               (scale * log2 e folded into one FFMA), write P as 16-bit
 //               pairs over the first 64 score columns (half h -> columns
 //               [32h, 32h + 32)) and keep fp32 partial sums (for LSE) and
@@ -74,9 +76,9 @@ struct FwdCfg {
   static constexpr uint32_t Q_OFF = 0;
   static constexpr uint32_t KV_OFF = 2 * TILE;
   static constexpr uint32_t BAR_OFF = KV_OFF + NSLOT * TILE;
-  // q_full[2] kv_full[N] kv_empty[N] s_full[2] p_full[4] mx_full[2] o_ready[2]
+  // q_full[2] kv_full[N] kv_empty[N] s_full[2] p_full[4] mx_full[8] o_ready[2]
   // pv_done[2] stats_ready[2] o_full[2] drain
-  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 4 + 2 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 4 + 8 + 2 + 2 + 2 + 2 + 1;
   // partial row maxima [tile][half][128] and the final partial sums
   // (l, lr)[tile][half][2][128], fp32
   static constexpr uint32_t XCH_OFF = (BAR_OFF + NBAR * 8 + 16 + 15) & ~15u;
@@ -135,8 +137,9 @@ __global__ void __launch_bounds__(768, 1)
   uint64_t* kv_empty = kv_full + C::NSLOT;
   uint64_t* s_full = kv_empty + C::NSLOT;  // [tile]: S ready (tensor core)
   uint64_t* p_full = s_full + 2;           // [tile * 2 + half]: P of 64 keys written (softmax)
-  uint64_t* mx_full = p_full + 4;          // [tile]: both partial row maxima published (softmax)
-  uint64_t* o_ready = mx_full + 2;         // [tile]: O ready for this step's P V (correction)
+  uint64_t* mx_full = p_full + 4;          // [tile * 4 + quarter]: both partial maxima of the
+                                           //   quarter's 32 rows published (its two softmax warps)
+  uint64_t* o_ready = mx_full + 8;         // [tile]: O ready for this step's P V (correction)
   uint64_t* pv_done = o_ready + 2;         // [tile]: one more P V product finished (tensor core)
   uint64_t* stats_ready = pv_done + 2;     // [tile]: final partial sums published (softmax)
   uint64_t* o_full = stats_ready + 2;      // [tile]: every P V product finished (tensor core)
@@ -152,8 +155,8 @@ __global__ void __launch_bounds__(768, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&mx_full[i], 256);
       mbar_init(&o_ready[i], 128);
+      for (int q = 0; q < 4; ++q) mbar_init(&mx_full[4 * i + q], 64);
       mbar_init(&pv_done[i], 1);
       mbar_init(&stats_ready[i], 256);
       mbar_init(&o_full[i], 1);
@@ -394,12 +397,13 @@ __global__ void __launch_bounds__(768, 1)
         }
         mx2[c] = fmax3(a, b, fmaxf(__uint_as_float(sv[c][30]), __uint_as_float(sv[c][31])));
       }
-      // swap partial maxima with the other half of the row (all 256
-      // threads of the tile arrive; the correction warpgroup reads them too)
+      // swap partial maxima with the other half of the row: only the two
+      // warps of these 32 rows arrive (and the correction warp of the same
+      // rows reads them too), so no warp waits for the tile's slowest one
       const float pm = fmaxf(mx2[0], mx2[1]);
       *my_max = pm;
-      mbar_arrive(&mx_full[t]);
-      ok = __all_sync(0xffffffffu, mbar_wait(&mx_full[t], j & 1, FWD_SITE_MX));
+      mbar_arrive(&mx_full[4 * t + (warp & 3)]);
+      ok = __all_sync(0xffffffffu, mbar_wait(&mx_full[4 * t + (warp & 3)], j & 1, FWD_SITE_MX));
       if (!ok) break;
       const float mx = fmaxf(pm, *other_max);
       // Exact running max: rescale whenever the row max grows, so the
@@ -478,7 +482,7 @@ __global__ void __launch_bounds__(768, 1)
       for (int t = 0; t < 2; ++t) {
         if (j >= (t ? n1 : n0)) continue;
         // this step's partial maxima -> the same running max the softmax keeps
-        ok = __all_sync(0xffffffffu, mbar_wait(&mx_full[t], j & 1, FWD_SITE_MX));
+        ok = __all_sync(0xffffffffu, mbar_wait(&mx_full[4 * t + (warp & 3)], j & 1, FWD_SITE_MX));
         if (!ok) break;
         const float mx = fmaxf(pmax_buf[(2 * t) * 128 + r], pmax_buf[(2 * t + 1) * 128 + r]);
         const float m = t ? m_row1 : m_row0;
