@@ -65,7 +65,7 @@ def flops(w):
 NCU_TRAFFIC = {
     "bwd_main": (289_130_957, "015da12a81d87b63e77598732a9fcbca3eca84d1bbd4ee8eb74bb88f2f4bc66f",
                  ("fa_bwd.cuh", "sm100.cuh")),
-    "fwd": (149_943_885, "60d40782546f254928a296b48e46227a32b0386512a60093b94047a7f3b88867",
+    "fwd": (151_631_642, "44bf43a5f4609a34b73445fd2c1ff632a5ceb5b5098a84206308e1354c97d38a",
             ("fa_fwd.cuh", "sm100.cuh")),
     # decode split kernel, B8 Hq32 Hkv8 L8192 D128 bf16, 2 splits merged in-kernel (mean of 13 launches)
     "decode": (268_978_708, "4696a7ff08d2327e8bf9a19eb0d9726cd3c9d323b54f6fb50c07502f9a1c391b",
