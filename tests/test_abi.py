@@ -87,6 +87,32 @@ def test_varlen_and_bwd_argument_errors(lib):
     assert fa.fa_bwd(*([A] * 9), 1, 1, 64, 48, 0.125, 1, 0, 0, A, need, None) == fa.api.FA_ERR_UNSUPPORTED
 
 
+def test_bwd_split_argument_errors(lib):
+    """fa_bwd_preprocess / fa_bwd_main / fa_bwd_finish refuse bad arguments
+    before launching anything (no GPU is touched here), with the same rules
+    as fa_bwd; fa_bwd_finish takes the deterministic flag of fa_bwd_main."""
+    A = 1 << 20
+    B, H, S, D, sc, bf = 1, 2, 300, 64, 0.125, fa.api.FA_BF16
+    need = fa.fa_bwd_workspace_size(B, H, S, D)
+    E, U = fa.api.FA_ERR_INVALID_ARG, fa.api.FA_ERR_UNSUPPORTED
+    pre = lambda ws=A, nb=need, d=D, dt=bf, o=A: fa.fa_bwd_preprocess(o, A, A, B, H, S, d, dt, ws, nb, None)
+    main = lambda ws=A, nb=need, d=D, dt=bf, q=A, det=1: fa.fa_bwd_main(q, A, A, A, A, A, B, H, S, d, sc, 1, dt, det,
+                                                                      ws, nb, None)
+    fin = lambda ws=A, nb=need, d=D, dt=bf, dq=A, s=sc, det=1: fa.fa_bwd_finish(dq, B, H, S, d, s, dt, det, ws, nb,
+                                                                               None)
+    for call in (pre, main, fin):
+        assert call(nb=need - 1) == E          # workspace too small
+        assert call(ws=A + 16) == E            # workspace not 256-byte aligned
+        assert call(ws=0) == E                 # no workspace
+        assert call(d=96) == U                 # head dim not built
+        assert call(dt=7) == E                 # unknown dtype
+    assert pre(o=A + 2) == E                   # misaligned O
+    assert main(q=0) == E                      # null Q
+    assert fin(dq=A + 8) == E                  # misaligned dQ
+    assert fin(s=float("nan")) == E            # bad scale
+    assert fa.fa_bwd_finish(A, 0, H, S, D, sc, bf, 1, 0, 0, None) == fa.api.FA_OK   # empty batch: nothing to do
+
+
 def test_missing_library_fails_loudly(tmp_path):
     saved = fa.api._lib
     fa.api._lib = None
