@@ -91,3 +91,26 @@ def test_bwd_varlen_deterministic_is_bitwise_repeatable(cuda_device):
     for a, b, name in zip(runs[0], nd, ("dQ", "dK", "dV")):
         check_grad(b, a, f"{name} atomic vs ordered")
     _check(t, True, 0.088, runs[0], [0, 3], "deterministic")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_varlen_deterministic_on_dirty_workspace(cuda_device, D, causal):
+    """Deterministic mode of a packed batch on a workspace full of 0x7F bytes
+    (3.4e38 as fp32): one-token, sub-tile, one-tile-plus-one and several-tile
+    sequences, so some query tiles have a single key tile (the second chain's
+    accumulator gets nothing there) and the packed rows of neighbouring
+    sequences share 32-row boxes; against the oracle, every sequence of every
+    head."""
+    lengths, H = [1, 130, 257, 64, 400], 3
+    t = _pack(lengths, H, D, "bf16", seed=11 + D + int(causal))
+    d = to_dev(t, cuda_device)
+    cu = t["cu_seqlens"].to(cuda_device)
+    L, scale = max(lengths), 1.0 / np.sqrt(D)
+    o, lse = fa.forward_varlen(d["q"], d["k"], d["v"], cu, L, causal, scale)
+    ws = torch.full((fa.fa_bwd_varlen_workspace_size(len(lengths), L, t["total"], H, D),), 0x7F, dtype=torch.uint8,
+                    device=cuda_device)
+    grads = fa.backward_varlen(d["q"], d["k"], d["v"], o, d["do"], lse, cu, L, causal, scale, deterministic=True,
+                               workspace=ws)
+    fa.check_device_error()
+    _check(t, causal, scale, grads, list(range(H)), f"deterministic dirty workspace D={D} causal={causal}")
