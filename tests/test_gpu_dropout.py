@@ -113,6 +113,26 @@ def test_dropout_deterministic_backward_is_bitwise_repeatable(cuda_device):
             assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("S,D,dtype,causal", [(1, 64, "bf16", True), (129, 128, "fp16", True),
+                                             (300, 64, "bf16", False), (257, 128, "bf16", False)])
+def test_dropout_deterministic_on_dirty_workspace_matches_oracle(cuda_device, S, D, dtype, causal):
+    """The dropout instances of the deterministic backward on a workspace
+    full of 0x7F bytes (3.4e38 as fp32), one tile and several, against the
+    oracle's dropout gradients."""
+    B, H, p, seed, offset = 1, 3, 0.25, 77, 5
+    q, k, v, do = _rand(B, H, S, D, dtype, seed=S * D)
+    scale = 1.0 / math.sqrt(D)
+    d = [x.to(cuda_device) for x in (q, k, v, do)]
+    o, lse = fa.forward(d[0], d[1], d[2], causal, scale, dropout_p=p, seed=seed, offset=offset)
+    ws = torch.full((fa.fa_bwd_workspace_size(B, H, S, D),), 0x7F, dtype=torch.uint8, device=cuda_device)
+    grads = fa.backward(d[0], d[1], d[2], o, d[3], lse, causal, scale, deterministic=True, workspace=ws,
+                        dropout_p=p, seed=seed, offset=offset)
+    fa.check_device_error()
+    g = oa.attention_backward_dropout(q, k, v, do, scale, causal, p, seed, offset)
+    for x, r, name in zip(grads, g, ("dQ", "dK", "dV")):
+        check_grad(x, r, f"deterministic dropout {name} S={S} D={D} {dtype} causal={causal}")
+
+
 def test_dropout_full_size_sampled(cuda_device):
     """B1 H32 S4096 D128 causal bf16, p = 0.1: O and LSE of the last head,
     the gradients of another, against the oracle."""
