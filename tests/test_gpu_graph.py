@@ -64,7 +64,7 @@ def test_forward_backward_graph_replays_bit_exactly(cuda_device, dropout_p):
             assert torch.equal(a, b), name
 
 
-@pytest.mark.parametrize("n_splits", [1, 2, 8])
+@pytest.mark.parametrize("n_splits", [1, 2, 8, 0])  # 0: balanced mode
 def test_decode_graph_replays_bit_exactly(cuda_device, n_splits):
     B, Hq, Hkv, L, D = 4, 16, 4, 2048, 128
     dev = cuda_device
